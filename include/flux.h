@@ -1,0 +1,182 @@
+/*
+ * flux.h -- C ABI of the B200 (sm_100a) hybrid-attention library "libflux".
+ *
+ * The library runs the hot path of Flux Attention ("Flux Attention: Context-Aware
+ * Hybrid Attention for Efficient LLMs Inference", arXiv 2604.07394):
+ *
+ *   flux_route      Layer Router (Figure 2): pool the query hidden states x_Q over
+ *                   the sequence boundaries (Figure 8), run a two-layer MLP and take
+ *                   a hard FA/SA decision per layer (Table 19 caption), written as a
+ *                   device-side bitmask.  The routing is decided once at prefill and
+ *                   reused by every decode step (Table 3, Flux Attention row).
+ *   flux_kv_append  write new K/V rows into a layer's contiguous KV cache.
+ *   flux_prefill    causal grouped-query attention of a prompt, Full Attention (FA)
+ *                   or streaming Sparse Attention (SA = attention-sink blocks plus a
+ *                   local window of KV blocks; Table 6, Figure 1 caption), chosen on
+ *                   the device from the layer's bit in the routing mask.
+ *   flux_decode     one autoregressive step of the same attention over the cache
+ *                   (split-KV partial softmax plus a combine pass).
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument that names tensor data is a DEVICE pointer owned by the
+ *     caller.  The library allocates and frees nothing; scratch space (the decode
+ *     workspace) is passed in by the caller.
+ *   - bf16 tensors are passed as uint16_t (raw bf16 bit patterns), row-major, densely
+ *     packed, with the layouts stated per call.  Base pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Every compute call is asynchronous on that stream and returns a flux_status.
+ *     Host-detected errors (bad arguments, unsupported shapes) return before any
+ *     launch.  Errors the device detects while running (a KV append past capacity, a
+ *     pipeline wait that ran out of time) never trap: the kernel skips the faulty
+ *     work, sets a bit in the library's device status word and returns; read and
+ *     clear that word with flux_get_device_status().
+ *   - Geometry: head_dim d in {64, 128}; SA block size in {64, 128}; sink and window
+ *     are multiples of the block size, window >= block.  Query head h reads KV head
+ *     h / (n_q_heads / n_kv_heads).  Softmax scale is 1/sqrt(d).
+ *   - SA visibility (block-granular reading of the streaming pattern): from query
+ *     position t (query block qb = t / block) key j is visible iff j <= t and its
+ *     block jb = j / block satisfies jb < sink/block or jb >= qb - window/block + 1.
+ *     FA visibility is j <= t.
+ */
+#ifndef FLUX_H
+#define FLUX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes of every call. */
+typedef enum flux_status {
+  FLUX_OK = 0,
+  FLUX_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shapes */
+  FLUX_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, block or group size */
+  FLUX_ERR_CAPACITY = 3,     /* host-visible capacity violation (n_new > capacity) */
+  FLUX_ERR_TIMEOUT = 4,      /* reported through the device status word only */
+  FLUX_ERR_CUDA = 5,         /* a CUDA runtime call or a kernel launch failed */
+  FLUX_ERR_WORKSPACE = 6     /* workspace missing or smaller than required */
+} flux_status;
+
+/* Bits of the device status word (flux_get_device_status). */
+#define FLUX_DEVICE_CAPACITY 0x1u /* a kv_append would pass the capacity; skipped */
+#define FLUX_DEVICE_TIMEOUT 0x2u  /* a pipeline wait ran out of time; output invalid */
+#define FLUX_DEVICE_BAD_LENGTH 0x4u /* seq_len < n_q in prefill, or seq_len > capacity */
+
+/* Attention geometry of one model; the same struct serves every layer. */
+typedef struct flux_attn_cfg {
+  int32_t n_layers;   /* layers covered by the routing mask (1..1024)             */
+  int32_t n_q_heads;  /* Hq                                                        */
+  int32_t n_kv_heads; /* Hkv; Hq % Hkv == 0; group Hq/Hkv in {1, 2, 4, 8}          */
+  int32_t head_dim;   /* d in {64, 128}                                            */
+  int32_t block;      /* SA block size in keys, 64 or 128                          */
+  int32_t sink;       /* SA attention-sink tokens, multiple of block, >= 0         */
+  int32_t window;     /* SA local window tokens, multiple of block, >= block       */
+} flux_attn_cfg;
+
+/* Layer Router parameters (Figure 2), bf16, (out, in) layout of a linear layer. */
+typedef struct flux_router_weights {
+  const uint16_t* w1; /* [rank][hidden]                                  */
+  const uint16_t* b1; /* [rank], or NULL for a zero bias                 */
+  const uint16_t* w2; /* [n_layers][rank]                                */
+  const uint16_t* b2; /* [n_layers], or NULL for a zero bias             */
+  int32_t hidden;     /* h, a multiple of 8, <= 16384                    */
+  int32_t rank;       /* r, 1..1024                                      */
+  int32_t n_layers;   /* 1..1024                                         */
+} flux_router_weights;
+
+/* Number of uint32 words per sequence in a routing mask: ceil(n_layers / 32). */
+int32_t flux_mask_words(int32_t n_layers);
+
+/*
+ * flux_route -- Layer Router (Figure 2; pooling window of Figure 8; hard decision of
+ * the per-layer soft FA probability, Table 19 caption).
+ *   xq       [batch][seq][hidden] bf16 query hidden states x_Q.
+ *   pool_len L: mean over the first ceil(L/2) and the last floor(L/2) tokens; L <= 0
+ *            or seq <= L pools every token.
+ *   z        = W2 relu(W1 mean(x_Q) + b1) + b2, accumulated in fp64 on the device.
+ *   fa_mask  [batch][flux_mask_words(n_layers)] uint32, written: bit (l % 32) of word
+ *            l / 32 is 1 iff z_l > tau (layer l runs FA), 0 for SA; unused bits 0.
+ *   logits   optional [batch][n_layers] double, the z values (NULL to skip).
+ * One kernel launch (a cluster of CTAs per sequence); reads only the pooled rows.
+ */
+int flux_route(const flux_router_weights* w, const uint16_t* xq, int32_t batch,
+               int32_t seq, int32_t pool_len, float tau, uint32_t* fa_mask,
+               double* logits, void* stream);
+
+/*
+ * flux_kv_append -- append n_new rows per sequence to one layer's KV cache.
+ *   k_cache, v_cache  [batch][n_kv_heads][capacity][head_dim] bf16 (read/write).
+ *   seq_len           [batch] int32 (read/write): rows are written at positions
+ *                     [seq_len[b], seq_len[b] + n_new) and seq_len[b] += n_new.
+ *   k_new, v_new      [batch][n_new][n_kv_heads][head_dim] bf16.
+ * A sequence with seq_len[b] + n_new > capacity is left untouched (rows and
+ * length) and FLUX_DEVICE_CAPACITY is set.  Two launches: copy, then length update.
+ */
+int flux_kv_append(const flux_attn_cfg* cfg, uint16_t* k_cache, uint16_t* v_cache,
+                   int32_t* seq_len, int32_t batch, int32_t capacity,
+                   const uint16_t* k_new, const uint16_t* v_new, int32_t n_new,
+                   void* stream);
+
+/*
+ * flux_prefill -- attention of n_q prompt queries per sequence for layer `layer`
+ * (Figure 2 routing; FA = causal dense path, SA = streaming sink + window path of
+ * Table 6), after their K/V rows have been appended.
+ *   fa_mask  [batch][flux_mask_words(n_layers)] from flux_route (or the caller).
+ *   q        [batch][n_q][n_q_heads][head_dim] bf16; query i of sequence b sits at
+ *            position t = seq_len[b] - n_q + i.
+ *   k_cache, v_cache, seq_len  as written by flux_kv_append (seq_len read only).
+ *   o        [batch][n_q][n_q_heads][head_dim] bf16, written.
+ * tcgen05 / TMEM tensor-core kernel fed by TMA; SA visits only the sink and window
+ * KV tiles.  seq_len[b] < n_q or > capacity sets FLUX_DEVICE_BAD_LENGTH and leaves
+ * that sequence's output unwritten.
+ */
+int flux_prefill(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                 const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                 const int32_t* seq_len, int32_t batch, int32_t capacity, int32_t n_q,
+                 uint16_t* o, void* stream);
+
+/* Bytes of device workspace flux_decode needs for this geometry and batch. */
+size_t flux_decode_workspace_size(const flux_attn_cfg* cfg, int32_t batch);
+
+/*
+ * flux_decode -- one decode step for layer `layer` (Table 3: the prefill route is
+ * reused), after the new token's K/V row has been appended.
+ *   q   [batch][n_q_heads][head_dim] bf16, the query at position seq_len[b] - 1.
+ *   o   [batch][n_q_heads][head_dim] bf16, written.
+ *   workspace  caller-owned device buffer of >= flux_decode_workspace_size() bytes
+ *              (split partial results; contents need no initialisation).
+ * Split-KV kernel (bulk-copy pipeline, 128-bit shared loads, warp-shuffle
+ * reductions) plus a combine kernel.  SA reads only the sink and window rows.
+ * seq_len[b] == 0 writes zeros; seq_len[b] > capacity sets FLUX_DEVICE_BAD_LENGTH.
+ */
+int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                const int32_t* seq_len, int32_t batch, int32_t capacity, uint16_t* o,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * flux_sa_block_ranges -- the SA key-block set of each query block, as the kernels
+ * compute it (streaming pattern of Table 6).  For query block qb (queries
+ * qb*block .. qb*block+block-1) the visible key blocks are [0, r[0]) united with
+ * [r[1], r[2]), where r = ranges + 3*qb.  ranges: [n_qblocks][3] int32 device memory.
+ */
+int flux_sa_block_ranges(const flux_attn_cfg* cfg, int32_t n_qblocks, int32_t* ranges,
+                         void* stream);
+
+/* Copy the device status word of the current device to *bits and clear it.
+ * Synchronises `stream` first. */
+int flux_get_device_status(void* stream, uint32_t* bits);
+
+/* Static English text for a flux_status value. */
+const char* flux_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t flux_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLUX_H */

@@ -1,0 +1,55 @@
+// Internal interface between the C-ABI layer (flux_api.cu) and the kernel files.
+// Arguments arrive here already validated; launchers return a cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace flux {
+
+struct AttnGeom {
+  int n_layers, mask_words, hq, hkv, head_dim, block, sink, window;
+};
+
+// ----- decode (split-KV + combine)
+constexpr int kDecMaxSplits = 64;   // splits per (sequence, KV head)
+constexpr int kDecMinChunk = 128;   // fewest keys per split before splitting further
+constexpr int kDecMaxBatch = 1024;
+
+size_t decode_workspace_bytes(const AttnGeom& g, int batch);
+
+cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                          const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                          const int32_t* seq_len, int batch, int capacity, uint16_t* o,
+                          void* workspace, unsigned* status, cudaStream_t stream);
+
+// ----- KV append
+cudaError_t launch_kv_append(const AttnGeom& g, uint16_t* k_cache, uint16_t* v_cache,
+                             int32_t* seq_len, int batch, int capacity, const uint16_t* k_new,
+                             const uint16_t* v_new, int n_new, unsigned* status,
+                             cudaStream_t stream);
+
+// ----- router
+constexpr int kRouterMaxHidden = 16384;
+constexpr int kRouterMaxRank = 1024;
+constexpr int kRouterMaxLayers = 1024;
+
+cudaError_t launch_route(const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                         const uint16_t* b2, int hidden, int rank, int n_layers,
+                         const uint16_t* xq, int batch, int seq, int pool_len, float tau,
+                         uint32_t* fa_mask, double* logits, cudaStream_t stream);
+
+// ----- prefill (tcgen05 / TMEM / TMA)
+cudaError_t launch_prefill(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                           const int32_t* seq_len, int batch, int capacity, int n_q, uint16_t* o,
+                           unsigned* status, cudaStream_t stream);
+
+// ----- SA block ranges (the block indices the kernels use)
+cudaError_t launch_sa_block_ranges(const AttnGeom& g, int n_qblocks, int32_t* ranges,
+                                   cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace flux

@@ -1,0 +1,74 @@
+// KV-cache append for the contiguous per-layer cache [B][Hkv][cap][d] (bf16).
+//
+// New rows arrive token-major ([B][n][Hkv][d], the layout a QKV projection writes)
+// and land head-major in the cache, so that every (sequence, KV head) keeps its keys
+// in one contiguous byte range -- the property the decode bulk copies and the prefill
+// TMA boxes rely on (the pages' "contiguous memory access" of layer-level routing).
+//
+// Two launches: the copy reads seq_len[b] as the write position; the second launch
+// advances seq_len[b], so no copy CTA can observe a half-updated length.  A sequence
+// that would pass the capacity is skipped and FLUX_DEVICE_CAPACITY is set.
+#include "flux_device.cuh"
+#include "flux_internal.h"
+
+namespace flux {
+namespace {
+
+__global__ void __launch_bounds__(256) kv_append_copy_kernel(
+    uint16_t* __restrict__ k_cache, uint16_t* __restrict__ v_cache,
+    const int32_t* __restrict__ seq_len, int capacity, const uint16_t* __restrict__ k_new,
+    const uint16_t* __restrict__ v_new, int n_new, int hkv, int chunks_per_row,
+    unsigned* status) {
+  const int b = blockIdx.y;
+  const int start = seq_len[b];
+  if (start < 0 || start + n_new > capacity) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, kStatusCapacity);
+    return;
+  }
+  const long long per_seq = (long long)n_new * hkv * chunks_per_row;
+  const size_t row_elems = size_t(chunks_per_row) * 8;
+  const uint4* ks = reinterpret_cast<const uint4*>(k_new) + size_t(b) * per_seq;
+  const uint4* vs = reinterpret_cast<const uint4*>(v_new) + size_t(b) * per_seq;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < per_seq;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int ch = int(i % chunks_per_row);
+    const long long rest = i / chunks_per_row;
+    const int kvh = int(rest % hkv);
+    const int tok = int(rest / hkv);
+    const size_t dst = ((size_t(b) * hkv + kvh) * capacity + start + tok) * row_elems + ch * 8;
+    const uint4 kv = __ldg(ks + i);
+    const uint4 vv = __ldg(vs + i);
+    *reinterpret_cast<uint4*>(k_cache + dst) = kv;
+    *reinterpret_cast<uint4*>(v_cache + dst) = vv;
+  }
+}
+
+__global__ void kv_append_advance_kernel(int32_t* seq_len, int batch, int capacity, int n_new) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= batch) return;
+  const int start = seq_len[b];
+  if (start >= 0 && start + n_new <= capacity) seq_len[b] = start + n_new;
+}
+
+}  // namespace
+
+cudaError_t launch_kv_append(const AttnGeom& g, uint16_t* k_cache, uint16_t* v_cache,
+                             int32_t* seq_len, int batch, int capacity, const uint16_t* k_new,
+                             const uint16_t* v_new, int n_new, unsigned* status,
+                             cudaStream_t stream) {
+  const int chunks = g.head_dim / 8;
+  const long long per_seq = (long long)n_new * g.hkv * chunks;
+  long long blocks = (per_seq + 255) / 256;
+  const long long cap_blocks = (long long)device_sm_count() * 16 / (batch > 0 ? batch : 1) + 1;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  if (blocks < 1) blocks = 1;
+  kv_append_copy_kernel<<<dim3(unsigned(blocks), batch), 256, 0, stream>>>(
+      k_cache, v_cache, seq_len, capacity, k_new, v_new, n_new, g.hkv, chunks, status);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  kv_append_advance_kernel<<<(batch + 127) / 128, 128, 0, stream>>>(seq_len, batch, capacity,
+                                                                     n_new);
+  return cudaGetLastError();
+}
+
+}  // namespace flux

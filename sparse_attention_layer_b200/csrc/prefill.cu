@@ -1,0 +1,628 @@
+// Causal GQA flash-attention prefill on the 5th-generation tensor cores (sm_100a),
+// for both routes of Flux Attention: Full Attention visits every KV tile up to the
+// diagonal, streaming Sparse Attention (Table 6: attention-sink blocks plus a local
+// window of blocks) visits only the sink tiles and the window tiles.  The route is
+// read on the device from the layer's bit of the router's mask (Figure 2).
+//
+// One CTA computes one 128-query tile of one query head.  Roles (192 threads):
+//   warps 0-3  softmax: thread i owns query row i; it reads its row of S = Q K^T from
+//              tensor memory (tcgen05.ld), masks boundary tiles, runs the online
+//              softmax in registers (log2 domain, a stale row maximum that is only
+//              raised when the new maximum exceeds it by more than 2^8, in which case
+//              the O row in tensor memory is rescaled), writes P as bf16 into shared
+//              memory in the 128-byte-swizzled K-major layout the MMA reads, and at
+//              the end normalises O and stores it.
+//   warp 4     TMA producer: the Q tile once, then K and V tiles into a 2-stage ring
+//              (cp.async.bulk.tensor, 128-byte swizzle, no cluster, no multicast).
+//   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two S buffers in
+//              tensor memory, then O += P_j V_j into the O accumulator; completion is
+//              signalled with tcgen05.commit on mbarriers.  The warp also allocates
+//              and frees the 512 tensor-memory columns (S0 | S1 | O).
+// S_{j+1} is issued before P_j V_j, so the tensor cores compute the next scores while
+// the softmax warps work on the current ones.
+//
+// Every mbarrier wait is bounded: on time-out the thread records FLUX_DEVICE_TIMEOUT
+// and leaves its loop; all roles meet at the final barrier, the producer first waits
+// for its copies in flight, and the tensor memory is always freed.
+#include <cuda.h>
+#include <math.h>
+
+#include "flux_device.cuh"
+#include "flux_internal.h"
+
+namespace flux {
+namespace {
+
+constexpr int BM = 128;  // query rows per tile (MMA M)
+constexpr int BN = 128;  // keys per KV tile (MMA N of Q K^T, MMA K of P V)
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSubBytes = 128 * 128;  // one 64-column swizzled sub-tile of 128 rows
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Smem {
+  static constexpr int NCH = D / 64;
+  static constexpr uint32_t tile = NCH * kSubBytes;  // Q tile or one K / V tile
+  static constexpr uint32_t off_q = 0;
+  static constexpr uint32_t off_k = off_q + tile;
+  static constexpr uint32_t off_v = off_k + kStages * tile;
+  static constexpr uint32_t off_p = off_v + kStages * tile;
+  static constexpr uint32_t off_bar = off_p + 2 * kSubBytes;
+  // q_full | k_full[S] | v_full[S] | kv_empty[S] | s_full[2] | p_full | o_done | mma_idle
+  static constexpr int n_bars = 1 + 3 * kStages + 2 + 3;
+  static constexpr uint32_t off_tmem = off_bar + n_bars * 8;
+  static constexpr uint32_t used = off_tmem + 16;
+  // 1 KB slack to align the base; at least 116 KB so that a second CTA (which would
+  // need its own 512 tensor-memory columns) never shares the SM.
+  static constexpr uint32_t bytes = (used + 1024) > 118784 ? (used + 1024) : 118784;
+};
+
+struct PrefillArgs {
+  const uint32_t* fa_mask;
+  int mask_words, layer;
+  const int32_t* seq_len;
+  int capacity, n_q, hq, hkv, block, sink, window, n_mtiles;
+  float scale_log2;
+  uint16_t* o;
+  unsigned* status;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 format (version 1).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;  // descriptor version for tcgen05
+  d |= uint64_t(2) << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 x bf16 -> fp32.
+constexpr uint32_t make_idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
+         (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+#define FLUX_TMEM_LD32(taddr, r)                                                               \
+  asm volatile(                                                                                \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "  \
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "  \
+      "%28, %29, %30, %31}, [%32];"                                                            \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),    \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),             \
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),          \
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),          \
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),          \
+        "=r"(r[31])                                                                            \
+      : "r"(taddr))
+
+#define FLUX_TMEM_ST32(taddr, r)                                                               \
+  asm volatile(                                                                                \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, " \
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "  \
+      "%28, %29, %30, %31, %32};" ::"r"(taddr),                                                \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),  \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),        \
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),      \
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),      \
+      "r"(r[29]), "r"(r[30]), "r"(r[31])                                                       \
+      : "memory")
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// ------------------------------------------------------------------ tile schedule
+
+// KV tiles of one query tile: tile index j < n0 is key tile j (the sink tiles); the
+// rest are key tiles w0 + (j - n0) (the window, up to the diagonal).  For FA n0 = 0
+// and w0 = 0.
+struct TilePlan {
+  int n0, w0, n_tiles;
+  int t_min, t_max;   // absolute positions of the tile's first and last real query
+  int win_lo_tmax;    // first window key of the last query (SA)
+  bool fa;
+};
+
+__device__ __forceinline__ int window_lo(int t, int block, int window) {
+  const int w = (t / block - window / block + 1) * block;
+  return w > 0 ? w : 0;
+}
+
+__device__ __forceinline__ TilePlan plan_tiles(const PrefillArgs& a, bool fa, int t_min, int t_max) {
+  TilePlan p;
+  p.fa = fa;
+  p.t_min = t_min;
+  p.t_max = t_max;
+  const int last = t_max / BN;
+  p.win_lo_tmax = window_lo(t_max, a.block, a.window);
+  if (fa) {
+    p.n0 = 0;
+    p.w0 = 0;
+    p.n_tiles = last + 1;
+    return p;
+  }
+  // union over the tile's queries: [0, min(sink, t_max+1)) U [window_lo(t_min), t_max]
+  const int sink_hi = a.sink < t_max + 1 ? a.sink : t_max + 1;
+  const int n_sink_tiles = (sink_hi + BN - 1) / BN;
+  const int w0 = window_lo(t_min, a.block, a.window) / BN;
+  if (w0 <= n_sink_tiles) {
+    p.n0 = 0;
+    p.w0 = 0;
+    p.n_tiles = last + 1;
+  } else {
+    p.n0 = n_sink_tiles;
+    p.w0 = w0;
+    p.n_tiles = n_sink_tiles + (last + 1 - w0);
+  }
+  return p;
+}
+
+__device__ __forceinline__ int tile_key0(const TilePlan& p, int j) {
+  return (j < p.n0 ? j : p.w0 + (j - p.n0)) * BN;
+}
+
+// True when some (query, key) pair of the tile is not visible.
+__device__ __forceinline__ bool tile_needs_mask(const TilePlan& p, int k0, int sink) {
+  if (k0 + BN - 1 > p.t_min) return true;  // crosses the causal diagonal / valid length
+  if (p.fa) return false;
+  if (k0 + BN <= sink) return false;       // wholly inside the sink
+  return k0 < p.win_lo_tmax;               // not wholly inside every query's window
+}
+
+// ------------------------------------------------------------------ the kernel
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+  using L = Smem<D>;
+  constexpr int NCH = L::NCH;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+
+  const uint32_t sQ = base + L::off_q;
+  const uint32_t sK = base + L::off_k;
+  const uint32_t sV = base + L::off_v;
+  const uint32_t sP = base + L::off_p;
+  const uint32_t bar0 = base + L::off_bar;
+  const uint32_t bar_q = bar0;
+  const uint32_t bar_kfull = bar0 + 8;                      // + 8 * stage
+  const uint32_t bar_vfull = bar0 + 8 * (1 + kStages);
+  const uint32_t bar_empty = bar0 + 8 * (1 + 2 * kStages);
+  const uint32_t bar_sfull = bar0 + 8 * (1 + 3 * kStages);  // + 8 * buffer
+  const uint32_t bar_pfull = bar0 + 8 * (3 + 3 * kStages);
+  const uint32_t bar_odone = bar0 + 8 * (4 + 3 * kStages);
+  const uint32_t bar_idle = bar0 + 8 * (5 + 3 * kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_tmem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int m_tile = a.n_mtiles - 1 - int(blockIdx.y);  // longest causal rows first
+  const int b = blockIdx.z;
+  const int kvh = h / (a.hq / a.hkv);
+
+  const int seq = a.seq_len[b];
+  if (seq < a.n_q || seq > a.capacity) {
+    if (tid == 0 && h == 0 && blockIdx.y == 0) atomicOr(a.status, kStatusBadLength);
+    return;
+  }
+  const int q_start = seq - a.n_q;
+  const int row0 = m_tile * BM;                    // first query index of the tile
+  const int rows = min(BM, a.n_q - row0);
+  const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
+  const TilePlan plan = plan_tiles(a, fa, q_start + row0, q_start + row0 + rows - 1);
+
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_kfull + 8 * s, 1);
+      mbar_init(bar_vfull + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_sfull + 8, 1);
+    mbar_init(bar_pfull, 4);
+    mbar_init(bar_odone, 1);
+    mbar_init(bar_idle, 1);
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_S0 = tmem;         // columns [0, 128)
+  const uint32_t tmem_O = tmem + 256;    // columns [256, 256 + D)
+
+  if (warp == kProducerWarp) {
+    // ---------------------------------------------------------------- TMA producer
+    int issued = 0;
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(bar_q, L::tile);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_4d(sQ + c * kSubBytes, &tmQ, c * 64, h, row0, b, bar_q);
+      const int kv_row = b * a.hkv + kvh;
+      for (int j = 0; j < plan.n_tiles; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (!mbar_wait(bar_empty + 8 * st, ph ^ 1, a.status)) break;
+        const int k0 = tile_key0(plan, j);
+        mbar_arrive_expect_tx(bar_kfull + 8 * st, L::tile);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_3d(sK + st * L::tile + c * kSubBytes, &tmK, c * 64, k0, kv_row,
+                      bar_kfull + 8 * st);
+        mbar_arrive_expect_tx(bar_vfull + 8 * st, L::tile);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_3d(sV + st * L::tile + c * kSubBytes, &tmV, c * 64, k0, kv_row,
+                      bar_vfull + 8 * st);
+        ++issued;
+      }
+      // wait for the copies in flight before the CTA may exit
+      mbar_wait(bar_q, 0, a.status);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        mbar_wait(bar_kfull + 8 * st, ph, a.status);
+        mbar_wait(bar_vfull + 8 * st, ph, a.status);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc(BM, BN, false, false);
+      constexpr uint32_t idesc_o = make_idesc(BM, D, false, true);
+      bool ok = mbar_wait(bar_q, 0, a.status);
+      // S_0
+      if (ok && plan.n_tiles > 0) {
+        ok = mbar_wait(bar_kfull, 0, a.status);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+            mma_bf16(tmem_S0, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + off, 16, 1024),
+                     idesc_s, kk > 0);
+          }
+          mma_commit(bar_sfull);
+        }
+      }
+      for (int j = 0; ok && j < plan.n_tiles; ++j) {
+        if (j + 1 < plan.n_tiles) {
+          const int jn = j + 1;
+          const int st = jn % kStages;
+          if (!mbar_wait(bar_kfull + 8 * st, (jn / kStages) & 1, a.status)) break;
+          tc_fence_after();
+          const uint32_t kb = sK + st * L::tile;
+          const uint32_t sbuf = tmem_S0 + (jn & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+            mma_bf16(sbuf, sw128_desc(sQ + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+                     idesc_s, kk > 0);
+          }
+          mma_commit(bar_sfull + 8 * (jn & 1));
+        }
+        const int st = j % kStages;
+        if (!mbar_wait(bar_pfull, j & 1, a.status)) break;
+        if (!mbar_wait(bar_vfull + 8 * st, (j / kStages) & 1, a.status)) break;
+        tc_fence_after();
+        const uint32_t vb = sV + st * L::tile;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+          mma_bf16(tmem_O, sw128_desc(sP + aoff, 16, 1024),
+                   sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o, (j > 0 || kk > 0));
+        }
+        mma_commit(bar_odone);
+        mma_commit(bar_empty + 8 * st);
+      }
+      // every MMA this thread issued has finished before tensor memory is freed
+      mma_commit(bar_idle);
+      mbar_wait(bar_idle, 0, a.status);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps
+    const int r = tid;                            // query row within the tile
+    const bool real_row = r < rows;
+    const int t = plan.t_min + (real_row ? r : rows - 1);
+    const int wl = window_lo(t, a.block, a.window);
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const float c = a.scale_log2;
+    float m_used = -INFINITY;  // scaled (log2) units
+    float l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < plan.n_tiles; ++j) {
+      if (!mbar_wait(bar_sfull + 8 * (j & 1), (j >> 1) & 1, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const int k0 = tile_key0(plan, j);
+      const bool masked = tile_needs_mask(plan, k0, a.sink);
+      const uint32_t srow = tmem_S0 + (j & 1) * 128 + lane_base;
+      uint32_t s[BN];
+#pragma unroll
+      for (int q = 0; q < BN / 32; ++q) {
+        uint32_t* sq = s + q * 32;
+        FLUX_TMEM_LD32(srow + q * 32, sq);
+      }
+      tmem_wait_ld();
+      if (masked) {
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          const int jk = k0 + i;
+          const bool vis = (jk <= t) && (plan.fa || jk < a.sink || jk >= wl);
+          if (!vis) s[i] = __float_as_uint(-INFINITY);
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+      const float m_tile = mx * c;
+      const bool raise = (m_used == -INFINITY) ? (m_tile > -INFINITY)
+                                               : (m_tile > m_used + kRescaleThreshold);
+      // P_{j-1} V_{j-1} must be complete before O is rescaled or P is overwritten
+      if (j > 0) {
+        if (!mbar_wait(bar_odone, (j - 1) & 1, a.status)) { ok = false; break; }
+        tc_fence_after();
+      }
+      float alpha = 1.f;
+      if (raise) {
+        alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_tile);
+        m_used = m_tile;
+        l_sum *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        const uint32_t orow = tmem_O + lane_base;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t ov[32];
+          FLUX_TMEM_LD32(orow + q * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          FLUX_TMEM_ST32(orow + q * 32, ov);
+        }
+        tmem_wait_st();
+      }
+      const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+      // P = exp2(S * c - m), row sum, bf16 into the swizzled K-major P tile
+#pragma unroll
+      for (int sb = 0; sb < 2; ++sb) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = sb * 64 + cc * 8 + 2 * e;
+            const float p0 = fast_exp2(fmaf(__uint_as_float(s[i]), c, -m_use));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(s[i + 1]), c, -m_use));
+            l_sum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          const uint32_t addr = sP + sb * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128 +
+                                ((cc ^ (r & 7)) << 4);
+          sts128(addr, pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      // keys past the valid length: zero their V rows (the cache there is unwritten)
+      if (k0 + BN > seq) {
+        const int st = j % kStages;
+        if (!mbar_wait(bar_vfull + 8 * st, (j / kStages) & 1, a.status)) { ok = false; break; }
+        if (k0 + r >= seq) {
+#pragma unroll
+          for (int cch = 0; cch < NCH; ++cch) {
+            const uint32_t vrow = sV + st * L::tile + cch * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) sts128(vrow + x * 16, 0u, 0u, 0u, 0u);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull);
+    }
+    // epilogue: O / l -> bf16 -> global
+    if (ok && plan.n_tiles > 0 && mbar_wait(bar_odone, (plan.n_tiles - 1) & 1, a.status)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_sum;
+      const uint32_t orow = tmem_O + lane_base;
+      uint16_t* dst = a.o + ((size_t(b) * a.n_q + row0 + r) * a.hq + h) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t ov[32];
+        FLUX_TMEM_LD32(orow + q * 32, ov);
+        tmem_wait_ld();
+        if (real_row) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[8 * x + 0]) * inv_l, __uint_as_float(ov[8 * x + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(ov[8 * x + 2]) * inv_l, __uint_as_float(ov[8 * x + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(ov[8 * x + 4]) * inv_l, __uint_as_float(ov[8 * x + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(ov[8 * x + 6]) * inv_l, __uint_as_float(ov[8 * x + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + q * 32 + x * 8) = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_prefill_t(const AttnGeom& g, const PrefillArgs& a, const uint16_t* q,
+                             const uint16_t* k_cache, const uint16_t* v_cache, int batch,
+                             cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  // Q: [B][n_q][Hq][D] as 4-D (D, Hq, n_q, B); box 64 x 1 x 128 x 1
+  const cuuint64_t qd[4] = {cuuint64_t(D), cuuint64_t(g.hq), cuuint64_t(a.n_q), cuuint64_t(batch)};
+  const cuuint64_t qs[3] = {cuuint64_t(D) * 2, cuuint64_t(g.hq) * D * 2,
+                            cuuint64_t(a.n_q) * g.hq * D * 2};
+  const cuuint32_t qbox[4] = {64, 1, BM, 1};
+  // K, V: [B][Hkv][cap][D] as 3-D (D, cap, B*Hkv); box 64 x 128 x 1
+  const cuuint64_t kd[3] = {cuuint64_t(D), cuuint64_t(a.capacity), cuuint64_t(batch) * g.hkv};
+  const cuuint64_t ks[2] = {cuuint64_t(D) * 2, cuuint64_t(a.capacity) * D * 2};
+  const cuuint32_t kbox[3] = {64, BN, 1};
+  if (!make_map(&mq, q, 4, qd, qs, qbox) || !make_map(&mk, k_cache, 3, kd, ks, kbox) ||
+      !make_map(&mv, v_cache, 3, kd, ks, kbox))
+    return cudaErrorInvalidValue;
+  const uint32_t smem = Smem<D>::bytes;
+  cudaError_t err =
+      cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return err;
+  const dim3 grid(g.hq, a.n_mtiles, batch);
+  prefill_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                           const int32_t* seq_len, int batch, int capacity, int n_q, uint16_t* o,
+                           unsigned* status, cudaStream_t stream) {
+  PrefillArgs a;
+  a.fa_mask = fa_mask;
+  a.mask_words = g.mask_words;
+  a.layer = layer;
+  a.seq_len = seq_len;
+  a.capacity = capacity;
+  a.n_q = n_q;
+  a.hq = g.hq;
+  a.hkv = g.hkv;
+  a.block = g.block;
+  a.sink = g.sink;
+  a.window = g.window;
+  a.n_mtiles = (n_q + BM - 1) / BM;
+  a.scale_log2 = float(1.4426950408889634 / sqrt(double(g.head_dim)));
+  a.o = o;
+  a.status = status;
+  if (a.n_mtiles > 65535) return cudaErrorInvalidValue;
+  if (g.head_dim == 128) return launch_prefill_t<128>(g, a, q, k_cache, v_cache, batch, stream);
+  if (g.head_dim == 64) return launch_prefill_t<64>(g, a, q, k_cache, v_cache, batch, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace flux

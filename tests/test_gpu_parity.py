@@ -1,0 +1,317 @@
+"""GPU parity: the CUDA path, called through the C ABI (ctypes binding), against the
+fp64 oracle on the same seeded inputs.
+
+Small cases span several 128-row tiles with ragged tails; full-size cases (the Llama
+and Qwen workloads, in the launch configuration the benchmark times) compare sampled
+rows the oracle computes one by one.  Router bits and SA block indices must match
+exactly; attention outputs within max-abs 2e-2 and relative L2 1e-2.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import flux_oracle as orc
+from sparse_attention_layer_b200 import configs, flux, inputs
+from sparse_attention_layer_b200.flux import AttnCfg
+from tests.gpu_cases import CacheCase, assert_close, f64, mask_words, oracle_layer, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    flux.flux_get_device_status()
+    yield
+
+
+def cfg_of(w: configs.Workload) -> AttnCfg:
+    return AttnCfg(w.n_layers, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.sink, w.window)
+
+
+# ------------------------------------------------------------------------- router
+
+
+def _route(w1, b1, w2, b2, xq, pool_len, tau):
+    batch, n_layers = xq.shape[0], w2.shape[0]
+    mask = torch.zeros(batch, (n_layers + 31) // 32, dtype=torch.int32, device="cuda")
+    logits = torch.zeros(batch, n_layers, dtype=torch.float64, device="cuda")
+    flux.flux_route(w1.cuda(), None if b1 is None else b1.cuda(), w2.cuda(),
+                    None if b2 is None else b2.cuda(), xq.cuda(), pool_len, tau, mask, logits)
+    torch.cuda.synchronize()
+    return mask.cpu(), logits.cpu().numpy()
+
+
+def _check_router(xq, w1, b1, w2, b2, pool_len, tau):
+    mask, z_gpu = _route(w1, b1, w2, b2, xq, pool_len, tau)
+    x64 = [t.float().numpy().astype(np.float64) for t in (xq, w1, b1, w2, b2)]
+    res = orc.router(*x64, pool_len, tau)
+    bound = orc.router_error_bound(*x64, pool_len)
+    # logits agree within the fp64 evaluation-order bound (both sides fp64)
+    assert (np.abs(z_gpu - res["logits"]) <= bound).all()
+    decided = np.abs(res["logits"] - tau) > bound
+    gpu_bits = ((mask.numpy().view(np.uint32)[:, np.arange(w2.shape[0]) // 32]
+                 >> (np.arange(w2.shape[0]) % 32)) & 1).astype(bool)
+    # unique decisions bit-exact; any undecidable one must follow the GPU's own logit
+    assert (gpu_bits[decided] == res["fa_bits"][decided]).all()
+    assert (gpu_bits[~decided] == (z_gpu[~decided] > tau)).all()
+    if decided.all():
+        assert (mask.numpy().view(np.uint32) == res["fa_mask"]).all()
+    return gpu_bits, res
+
+
+def test_router_toy_golden():
+    g = json.load(open(os.path.join(GOLDEN, "router_toy.json")))
+    pad = 8  # the library wants hidden % 8 == 0: zero columns leave the logits unchanged
+    xq = torch.zeros(1, 4, pad)
+    xq[:, :, :4] = torch.tensor(g["xq"], dtype=torch.float32)
+    w1 = torch.zeros(2, pad)
+    w1[:, :4] = torch.tensor(g["w1"], dtype=torch.float32)
+    b1 = torch.tensor(g["b1"]); w2 = torch.tensor(g["w2"]); b2 = torch.tensor(g["b2"])
+    bf = lambda t: t.to(torch.bfloat16)  # noqa: E731
+    for case in g["cases"]:
+        mask, z = _route(bf(w1), bf(b1), bf(w2), bf(b2), bf(xq), case["pool_len"], g["tau"])
+        assert np.allclose(z, case["logits"], atol=1e-9)
+        assert mask.numpy().view(np.uint32).tolist() == case["mask_words"]
+
+
+@pytest.mark.parametrize("pool_len", [100, 0, 7])
+def test_router_tiny(pool_len):
+    w = configs.TINY
+    xq = inputs.normal_bf16((2, w.seq, w.router_hidden), inputs.layer_seed(w.data_seed, 0, inputs.XQ))
+    w1, b1, w2, b2 = inputs.router_weights(w.router_hidden, w.router_rank, w.n_layers, w.router_seed)
+    _check_router(xq, w1, b1, w2, b2, pool_len, w.tau)
+
+
+def test_router_nonzero_bias_and_threshold():
+    xq = inputs.normal_bf16((3, 300, 256), 77)
+    w1 = inputs.normal_bf16((40, 256), 78, std=0.05)
+    w2 = inputs.normal_bf16((37, 40), 79, std=0.05)  # 37 layers: two mask words
+    b1 = inputs.normal_bf16((40,), 80, std=0.01)
+    b2 = inputs.normal_bf16((37,), 81, std=0.01)
+    _check_router(xq, w1, b1, w2, b2, 100, 0.003)
+
+
+@pytest.mark.parametrize("name", ["llama31_8b_prefill_8k", "qwen3_4b_prefill_128k"])
+def test_router_full_size(name):
+    w = configs.ALL[name]
+    seeds = json.load(open(os.path.join(GOLDEN, "router_seeds.json")))[name]
+    xq = inputs.normal_bf16((w.batch, w.seq, w.router_hidden),
+                            inputs.layer_seed(w.data_seed, 0, inputs.XQ))
+    w1, b1, w2, b2 = inputs.router_weights(w.router_hidden, w.router_rank, w.n_layers,
+                                           seeds["router_seed"])
+    bits, res = _check_router(xq, w1, b1, w2, b2, w.pool_len, w.tau)
+    assert bits[0].astype(int).tolist() == seeds["fa_bits"]
+    assert int((~bits).sum()) == w.target_sa_layers
+
+
+# ------------------------------------------------------------------ SA block indices
+
+
+@pytest.mark.parametrize("block,sink,window", [(64, 64, 256), (128, 128, 2048), (128, 128, 4096),
+                                               (64, 0, 64), (128, 256, 128), (64, 128, 256)])
+def test_sa_block_ranges_exact(block, sink, window):
+    cfg = AttnCfg(2, 8, 2, 64, block, sink, window)
+    n_qb = 80
+    ranges = torch.zeros(n_qb, 3, dtype=torch.int32, device="cuda")
+    flux.flux_sa_block_ranges(cfg, n_qb, ranges)
+    r = ranges.cpu().numpy()
+    for qb in range(n_qb):
+        got = set(range(0, r[qb, 0])) | set(range(r[qb, 1], r[qb, 2]))
+        want = orc.sa_visible_key_blocks(qb, qb + 1, block, sink, window)
+        assert got == want, (qb, r[qb].tolist(), sorted(want))
+
+
+# ------------------------------------------------------------------------ KV append
+
+
+def test_kv_append_exact_and_capacity():
+    cfg = AttnCfg(2, 8, 2, 64, 64, 64, 256)
+    batch, cap = 3, 40
+    k = torch.zeros(batch, 2, cap, 64, dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros_like(k)
+    seq = torch.tensor([0, 30, 38], dtype=torch.int32, device="cuda")
+    kn = inputs.normal_bf16((batch, 5, 2, 64), 5)
+    vn = inputs.normal_bf16((batch, 5, 2, 64), 6)
+    flux.flux_kv_append(cfg, k, v, seq, kn.cuda(), vn.cuda())
+    assert flux.flux_get_device_status() == flux.FLUX_DEVICE_CAPACITY
+    k2, v2, s2, over = orc.kv_append(np.zeros((batch, 2, cap, 64)), np.zeros((batch, 2, cap, 64)),
+                                     np.array([0, 30, 38]), f64(kn), f64(vn))
+    assert seq.cpu().tolist() == s2.tolist() and over.tolist() == [False, False, True]
+    assert np.array_equal(f64(k), k2) and np.array_equal(f64(v), v2)
+    # bit-exact copy, including the byte patterns
+    assert torch.equal(k[1, :, 30:35].cpu().view(torch.int16), kn[1].transpose(0, 1).view(torch.int16))
+
+
+# --------------------------------------------------------------------------- decode
+
+
+def _decode_case(cfg, ctx, fa_per_seq, steps, seed, capacity=None, layer=0):
+    batch = len(ctx)
+    cap = capacity or (max(ctx) + steps + 8)
+    case = CacheCase(cfg, ctx, cap, seed)
+    fa_rows = [[layer] if fa else [] for fa in fa_per_seq]
+    mask = mask_words(batch, cfg.n_layers, fa_rows).cuda()
+    ws = torch.empty(flux.flux_decode_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    for step in range(steps):
+        kn = inputs.normal_bf16((batch, 1, cfg.n_kv_heads, cfg.head_dim), seed * 31 + step * 3 + 1)
+        vn = inputs.normal_bf16((batch, 1, cfg.n_kv_heads, cfg.head_dim), seed * 31 + step * 3 + 2)
+        q = inputs.normal_bf16((batch, cfg.n_q_heads, cfg.head_dim), seed * 31 + step * 3 + 3)
+        case.append(kn, vn)
+        o = torch.empty(batch, cfg.n_q_heads, cfg.head_dim, dtype=torch.bfloat16, device="cuda")
+        flux.flux_decode(cfg, layer, mask, q.cuda(), case.k, case.v, case.seq_len, o, ws)
+        torch.cuda.synchronize()
+        want = oracle_layer(case, q[:, None], fa_per_seq)[:, 0]
+        assert_close(f64(o), want, f"decode step {step}")
+    assert flux.flux_get_device_status() == 0
+
+
+def test_decode_tiny_config():
+    """Tiny workload: 1024-token context, layer 0 FA and layer 1 SA, 16 decode steps."""
+    w = configs.TINY
+    cfg = cfg_of(w)
+    for layer, fa in ((0, True), (1, False)):
+        _decode_case(cfg, [w.seq], [fa], w.decode_steps, seed=100 + layer, layer=layer)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+def test_decode_groups_and_head_dims(d, group):
+    cfg = AttnCfg(3, 2 * group, 2, d, 64, 64, 192)
+    _decode_case(cfg, [700, 1, 64, 333, 4000], [True, False, True, False, False], 2,
+                 seed=7 + group + d, layer=2)
+
+
+def test_decode_ragged_edges():
+    """Contexts shorter than the sink, exactly one block, one key past the window."""
+    cfg = AttnCfg(1, 8, 2, 128, 128, 128, 256)
+    ctx = [0, 5, 127, 128, 383, 384, 385, 9000]
+    _decode_case(cfg, ctx, [False] * len(ctx), 1, seed=3)
+    _decode_case(cfg, ctx, [True] * len(ctx), 1, seed=4)
+
+
+def test_decode_empty_sequence_writes_zeros():
+    cfg = AttnCfg(1, 4, 1, 64, 64, 64, 64)
+    k = torch.zeros(2, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    seq = torch.tensor([0, 0], dtype=torch.int32, device="cuda")
+    mask = torch.zeros(2, 1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(flux.flux_decode_workspace_size(cfg, 2), dtype=torch.uint8, device="cuda")
+    o = torch.full((2, 4, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    q = torch.ones(2, 4, 64, dtype=torch.bfloat16, device="cuda")
+    flux.flux_decode(cfg, 0, mask, q, k, k, seq, o, ws)
+    torch.cuda.synchronize()
+    assert (o == 0).all()
+
+
+def test_decode_bad_length_flag():
+    cfg = AttnCfg(1, 4, 1, 64, 64, 64, 64)
+    k = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    seq = torch.tensor([17], dtype=torch.int32, device="cuda")  # past capacity 16
+    mask = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(flux.flux_decode_workspace_size(cfg, 1), dtype=torch.uint8, device="cuda")
+    o = torch.empty(1, 4, 64, dtype=torch.bfloat16, device="cuda")
+    flux.flux_decode(cfg, 0, mask, torch.ones_like(o), k, k, seq, o, ws)
+    assert flux.flux_get_device_status() & flux.FLUX_DEVICE_BAD_LENGTH
+
+
+# -------------------------------------------------------------------------- prefill
+
+
+def _prefill_case(cfg, q_start, n_q, fa_per_seq, seed, layer=0, rows=None, heads=None,
+                  capacity=None):
+    batch = len(q_start)
+    cap = capacity or (max(q_start) + n_q + 5)
+    case = CacheCase(cfg, q_start, cap, seed)
+    kn = inputs.normal_bf16((batch, n_q, cfg.n_kv_heads, cfg.head_dim), seed * 17 + 1)
+    vn = inputs.normal_bf16((batch, n_q, cfg.n_kv_heads, cfg.head_dim), seed * 17 + 2)
+    q = inputs.normal_bf16((batch, n_q, cfg.n_q_heads, cfg.head_dim), seed * 17 + 3)
+    case.append(kn, vn)
+    fa_rows = [[layer] if fa else [] for fa in fa_per_seq]
+    mask = mask_words(batch, cfg.n_layers, fa_rows).cuda()
+    o = torch.empty(batch, n_q, cfg.n_q_heads, cfg.head_dim, dtype=torch.bfloat16, device="cuda")
+    flux.flux_prefill(cfg, layer, mask, q.cuda(), case.k, case.v, case.seq_len, o)
+    torch.cuda.synchronize()
+    assert flux.flux_get_device_status() == 0
+    want = oracle_layer(case, q, fa_per_seq, rows=rows, heads=heads)
+    got = o.cpu()
+    if rows is not None:
+        got = got[:, torch.as_tensor(rows)]
+    if heads is not None:
+        got = got[:, :, torch.as_tensor(heads)]
+    return assert_close(f64(got), want, "prefill")
+
+
+def test_prefill_tiny_config():
+    """Tiny workload prefill: 1024 tokens, layer 0 FA, layer 1 SA (block 64)."""
+    w = configs.TINY
+    cfg = cfg_of(w)
+    _prefill_case(cfg, [0], w.seq, [True], seed=200, layer=0)
+    _prefill_case(cfg, [0], w.seq, [False], seed=201, layer=1)
+
+
+@pytest.mark.parametrize("fa", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_ragged_tail(fa, d):
+    cfg = AttnCfg(1, 4, 2, d, 128, 128, 256)
+    _prefill_case(cfg, [0], 1000, [fa], seed=300 + d + fa)   # 1000 = 7 tiles + 104 rows
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_prefill_chunked_and_mixed_batch(block):
+    """Queries after an existing prefix (chunked prefill), per-sequence routes, ragged
+    lengths in one batch."""
+    cfg = AttnCfg(2, 8, 2, 128, block, block, 4 * block)
+    _prefill_case(cfg, [0, 300, 1024, 77], 700, [False, True, False, True], seed=400 + block,
+                  layer=1)
+
+
+@pytest.mark.parametrize("group", [1, 2, 8])
+def test_prefill_groups(group):
+    cfg = AttnCfg(1, 2 * group, 2, 64, 64, 0, 128)   # no sink
+    _prefill_case(cfg, [0], 600, [False], seed=500 + group)
+
+
+def test_prefill_short_sequences():
+    cfg = AttnCfg(1, 4, 1, 128, 128, 128, 128)
+    for n_q in (1, 2, 127, 128, 129):
+        _prefill_case(cfg, [0], n_q, [False], seed=600 + n_q)
+        _prefill_case(cfg, [0], n_q, [True], seed=700 + n_q)
+
+
+# ------------------------------------------------------------ full-size workloads
+
+
+@pytest.mark.parametrize("fa", [True, False])
+def test_prefill_llama_full_size(fa):
+    """Llama-3.1-8B shape, 8192-token prompt, one FA and one SA layer; sampled rows."""
+    w = configs.LLAMA_PREFILL
+    cfg = cfg_of(w)
+    rows = sample_rows(w.seq, 0, cfg, 40, seed=1)
+    _prefill_case(cfg, [0], w.seq, [fa], seed=800 + fa, rows=rows, heads=[0, 5, 17, 31],
+                  capacity=w.seq)
+
+
+@pytest.mark.parametrize("fa", [True, False])
+def test_prefill_qwen_full_size(fa):
+    """Qwen3-4B shape, 131072-token prompt, SA window 4096; sampled rows."""
+    w = configs.QWEN_PREFILL
+    cfg = cfg_of(w)
+    rows = sample_rows(w.seq, 0, cfg, 16, seed=2)
+    _prefill_case(cfg, [0], w.seq, [fa], seed=900 + fa, rows=rows, heads=[0, 31],
+                  capacity=w.seq)
+
+
+def test_decode_llama_full_size():
+    """Llama-3.1-8B decode: 16 sequences at 32768 context, FA and SA layers."""
+    w = configs.LLAMA_DECODE
+    cfg = cfg_of(w)
+    ctx = [w.seq] * w.batch
+    _decode_case(cfg, ctx, [True] * w.batch, 1, seed=1000, capacity=w.capacity(), layer=3)
+    _decode_case(cfg, ctx, [False] * w.batch, 2, seed=1001, capacity=w.capacity(), layer=4)
