@@ -1,0 +1,578 @@
+"""Benchmark of the hybrid-attention hot path (Flux Attention: layer router + FA/SA
+prefill + FA/SA decode) on B200.
+
+Main line (`value`): decode tokens/s of the Llama-3.1-8B attention shape serving 16
+sequences at a 32768-token context, 32 layers of which a fixed seeded 16 run SA
+(sink 128 + window 2048, block 128).  One step = one decode token for every sequence:
+per layer a KV append and an FA- or SA-routed split-KV decode.  The same run also
+times the prefill phase (router + 32 x (KV append + FA/SA prefill) of an 8192-token
+Llama-shaped prompt with router-chosen routes) and the decode step at every SA-layer
+fraction of the routing mix.  Protocol: W warm-up then K timed steps (default 10 and
+50), CUDA events on the launching stream, barrier + synchronize around the timed
+region, max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead, on a bounded
+sample of the same decode workload, and prints the same metric.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flux|reference]
+Multi-GPU (replicas, no data-path collective):
+  python -m torch.distributed.run --nproc-per-node N --master-addr 127.0.0.1 bench.py --gpus N
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "hybrid-attn prefill & decode tokens/s at 32K ctx; % of tensor/HBM roofline"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------ helpers
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"flux_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.remove(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if world != n_gpus:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        import numpy  # noqa: F401
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # noqa: BLE001
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- workloads
+
+
+def decode_geometry():
+    from sparse_attention_layer_b200 import configs
+    from sparse_attention_layer_b200.flux import AttnCfg
+    w = configs.LLAMA_DECODE
+    cfg = AttnCfg(w.n_layers, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.sink, w.window)
+    return w, cfg
+
+
+def decode_bytes_per_layer(w, cfg, T: int, fa: bool) -> int:
+    """Algorithmic bytes of one decode launch: K and V rows of every visible key plus
+    q in and o out, for all sequences."""
+    if fa:
+        n_vis = T
+    else:
+        t = T - 1
+        qb = t // cfg.block
+        win_lo = max(0, (qb - cfg.window // cfg.block + 1) * cfg.block)
+        n_vis = (T - win_lo) + min(cfg.sink, win_lo)
+    kv = 2 * 2 * w.batch * cfg.n_kv_heads * cfg.head_dim * n_vis
+    qo = 2 * 2 * w.batch * cfg.n_q_heads * cfg.head_dim
+    return kv + qo
+
+
+def prefill_flops_per_layer(cfg, S: int, fa: bool) -> float:
+    """Algorithmic flops of one prefill launch (batch 1): 4 d Hq per visible pair."""
+    total = 0
+    for t in range(S):
+        if fa:
+            total += t + 1
+        else:
+            qb = t // cfg.block
+            win_lo = max(0, (qb - cfg.window // cfg.block + 1) * cfg.block)
+            total += (t + 1 - win_lo) + min(cfg.sink, win_lo)
+    return 4.0 * cfg.head_dim * cfg.n_q_heads * total
+
+
+class DecodeBench:
+    """Llama-shape decode at 32K context: 32 layers of KV cache resident in HBM."""
+
+    def __init__(self, seed: int):
+        from sparse_attention_layer_b200 import configs, inputs
+        from sparse_attention_layer_b200.runtime import HybridAttention
+        self.w, self.cfg = decode_geometry()
+        w, cfg = self.w, self.cfg
+        self.model = HybridAttention(cfg, w.batch, w.capacity(), "cuda")
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        for c in self.model.caches:
+            c.k[:, :, :w.seq].normal_(generator=gen)
+            c.v[:, :, :w.seq].normal_(generator=gen)
+        self.ctx = w.seq
+        self.sa_layers = inputs.fixed_sa_layers(w.n_layers, w.target_sa_layers,
+                                                configs.LLAMA_DECODE_MASK_SEED)
+        self.set_sa_layers(self.sa_layers)
+        L, B = w.n_layers, w.batch
+        self.q = torch.randn(L, B, cfg.n_q_heads, cfg.head_dim, device="cuda",
+                             generator=gen).to(torch.bfloat16)
+        self.k_new = torch.randn(L, B, 1, cfg.n_kv_heads, cfg.head_dim, device="cuda",
+                                 generator=gen).to(torch.bfloat16)
+        self.v_new = torch.randn(L, B, 1, cfg.n_kv_heads, cfg.head_dim, device="cuda",
+                                 generator=gen).to(torch.bfloat16)
+        self.o = torch.empty(L, B, cfg.n_q_heads, cfg.head_dim, dtype=torch.bfloat16,
+                             device="cuda")
+
+    def set_sa_layers(self, sa_layers):
+        from sparse_attention_layer_b200 import inputs
+        bits = inputs.fa_bits_from_sa_layers(self.w.batch, self.w.n_layers, sa_layers)
+        self.fa = [bool(bits[0, i]) for i in range(self.w.n_layers)]
+        self.model.set_mask(inputs.pack_bits_u32(bits).cuda())
+
+    def reset(self):
+        for c in self.model.caches:
+            c.seq_len.fill_(self.ctx)
+
+    def step(self, fa_events=None):
+        """One decode token for every sequence through all layers.  With fa_events, the
+        flux_decode call of every FA layer is bracketed by CUDA events."""
+        from sparse_attention_layer_b200 import flux
+        m = self.model
+        for layer in range(self.w.n_layers):
+            c = m.caches[layer]
+            flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, self.k_new[layer],
+                                self.v_new[layer])
+            timed = fa_events is not None and self.fa[layer]
+            if timed:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            flux.flux_decode(self.cfg, layer, m.fa_mask, self.q[layer], c.k, c.v, c.seq_len,
+                             self.o[layer], m.workspace)
+            if timed:
+                e1.record()
+                fa_events.append((e0, e1))
+
+    launches_per_step = property(lambda self: self.w.n_layers * 4)  # append 2 + decode 2
+
+
+class PrefillBench:
+    """Llama-shape prefill: router on x_Q, then 32 x (KV append + FA/SA prefill), S=8192."""
+
+    def __init__(self, seed: int):
+        from sparse_attention_layer_b200 import configs, inputs
+        from sparse_attention_layer_b200.flux import AttnCfg
+        from sparse_attention_layer_b200.runtime import HybridAttention
+        w = configs.LLAMA_PREFILL
+        self.w = w
+        self.cfg = AttnCfg(w.n_layers, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.sink,
+                           w.window)
+        self.model = HybridAttention(self.cfg, w.batch, w.seq, "cuda")
+        w1, b1, w2, b2 = inputs.router_weights(w.router_hidden, w.router_rank, w.n_layers,
+                                               w.router_seed)
+        self.router = [t.cuda() for t in (w1, b1, w2, b2)]
+        self.xq = inputs.normal_bf16((w.batch, w.seq, w.router_hidden),
+                                     inputs.layer_seed(w.data_seed, 0, inputs.XQ)).cuda()
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        L, B, S = w.n_layers, w.batch, w.seq
+        self.q = torch.randn(L, B, S, w.n_q_heads, w.head_dim, device="cuda",
+                             generator=gen).to(torch.bfloat16)
+        self.k = torch.randn(L, B, S, w.n_kv_heads, w.head_dim, device="cuda",
+                             generator=gen).to(torch.bfloat16)
+        self.v = torch.randn(L, B, S, w.n_kv_heads, w.head_dim, device="cuda",
+                             generator=gen).to(torch.bfloat16)
+        self.o = torch.empty(B, S, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+        # route once to learn the mask (the timed steps route again)
+        self.model.route(*self.router, self.xq, w.pool_len, w.tau)
+        words = self.model.fa_mask.cpu()[0]
+        self.fa = [bool((int(words[i // 32]) >> (i % 32)) & 1) for i in range(L)]
+
+    def reset(self):
+        for c in self.model.caches:
+            c.seq_len.zero_()
+
+    def step(self, fa_events=None, router_events=None):
+        from sparse_attention_layer_b200 import flux
+        m, w = self.model, self.w
+        if router_events is not None:
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+        m.route(*self.router, self.xq, w.pool_len, w.tau)
+        if router_events is not None:
+            e1.record(); router_events.append((e0, e1))
+        for layer in range(w.n_layers):
+            c = m.caches[layer]
+            flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, self.k[layer], self.v[layer])
+            if fa_events is not None and self.fa[layer]:
+                e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            flux.flux_prefill(self.cfg, layer, m.fa_mask, self.q[layer], c.k, c.v, c.seq_len,
+                              self.o)
+            if fa_events is not None and self.fa[layer]:
+                e1.record(); fa_events.append((e0, e1))
+
+    launches_per_step = property(lambda self: 1 + self.w.n_layers * 3)  # route 1, append 2, prefill 1
+
+
+def elapsed_ms(pairs):
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+# ---------------------------------------------------------------- CPU baseline
+
+
+def cpu_oracle_decode_sample(n_seq: int = 1, seed: int = 5):
+    """Time the fp64 oracle on one decode step of n_seq sequences of the 32K decode
+    workload, for one FA and one SA layer; returns seconds per layer-step per sequence."""
+    import numpy as np
+
+    from oracle import flux_oracle as orc
+    from sparse_attention_layer_b200 import inputs
+    w, cfg = decode_geometry()
+    T = w.seq + 1
+    shape = (n_seq, cfg.n_kv_heads, T, cfg.head_dim)
+    kc = inputs.normal_bf16(shape, seed).float().numpy().astype(np.float64)
+    vc = inputs.normal_bf16(shape, seed + 1).float().numpy().astype(np.float64)
+    q = inputs.normal_bf16((n_seq, cfg.n_q_heads, cfg.head_dim), seed + 2).float().numpy().astype(np.float64)
+    lens = np.full(n_seq, T)
+    out = {}
+    for fa in (True, False):
+        t0 = time.perf_counter()
+        orc.decode_attention(q, kc, vc, lens, np.full(n_seq, fa), cfg.block, cfg.sink, cfg.window)
+        out[fa] = (time.perf_counter() - t0) / n_seq
+    return out
+
+
+def cpu_baseline_decode_tok_s(w, n_sa, n_seq=2):
+    per = cpu_oracle_decode_sample(n_seq)
+    per_seq_step = (w.n_layers - n_sa) * per[True] + n_sa * per[False]
+    return 1.0 / per_seq_step, per
+
+
+# ---------------------------------------------------------------------- runs
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host cores, on bounded samples of the decode workload."""
+    if rank != 0:
+        return
+    from sparse_attention_layer_b200 import configs, inputs
+    w, cfg = decode_geometry()
+    sa = inputs.fixed_sa_layers(w.n_layers, w.target_sa_layers, configs.LLAMA_DECODE_MASK_SEED)
+    for _ in range(args.warmup):
+        cpu_oracle_decode_sample(1)
+    times = []
+    for _ in range(args.steps):
+        per = cpu_oracle_decode_sample(1)
+        times.append((w.n_layers - len(sa)) * per[True] + len(sa) * per[False])
+    per_seq_step = statistics.mean(times)
+    value = 1.0 / per_seq_step
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_seq_step * 1e3 * w.batch, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": decode_config(w, cfg, sa),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: one decode token of 1 of the 16 sequences at "
+                                   "32768 context, one FA and one SA layer, scaled to 16 FA + "
+                                   "16 SA layers; a batch of 16 costs 16x (sequences are "
+                                   "independent)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def decode_config(w, cfg, sa_layers):
+    return {"workload": "llama3.1-8b-shape hybrid attention decode, 16 sequences at 32768 "
+                        "context, 32 layers (16 FA + 16 SA, fixed seeded mask)",
+            "batch": w.batch, "context": w.seq, "n_layers": w.n_layers,
+            "q_heads": cfg.n_q_heads, "kv_heads": cfg.n_kv_heads, "head_dim": cfg.head_dim,
+            "sa_layers": len(sa_layers), "sink": cfg.sink, "window": cfg.window,
+            "block": cfg.block, "parallelism": "replicas (one independent model per GPU)",
+            "l2": "no flush needed: each step streams ~37 GB of KV, far above the 126 MB L2"}
+
+
+def run_flux(args, world, rank, local):
+    from sparse_attention_layer_b200 import flux
+    peaks, peak_kind = load_peaks()
+    db = DecodeBench(seed=1234 + rank)
+    w, cfg = db.w, db.cfg
+    sa_layers = list(db.sa_layers)
+
+    # ---------------- decode: main metric
+    db.reset()
+    for _ in range(args.warmup):
+        db.step()
+    db.reset()
+    sampler = ClockSampler(local)
+    barrier(world)
+    sampler.start()
+    fa_events = []
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    start.record()
+    for _ in range(args.steps):
+        db.step(fa_events=fa_events)
+    end.record()
+    barrier(world)
+    clocks = sampler.stop()
+    st = flux.flux_get_device_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} after the decode steps")
+    t_ms = max_over_ranks(start.elapsed_time(end), world)
+    ms_step = t_ms / args.steps
+    value = world * w.batch * args.steps / (t_ms / 1e3)
+    fa_ms = elapsed_ms(fa_events)
+    # the timed steps run contexts 32769 .. 32768 + K; take the mean context
+    T_mean = w.seq + (args.steps + 1) / 2.0
+    fa_bytes = decode_bytes_per_layer(w, cfg, int(round(T_mean)), True)
+    achieved = fa_bytes / (statistics.mean(fa_ms) / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "flux_decode (split-KV + combine), FA layers",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_kind": f"{peak_kind} hbm_gbs",
+                "traffic": None, "launch_ms": statistics.mean(fa_ms),
+                "algorithmic_bytes_per_launch": fa_bytes}
+    sa_bytes = decode_bytes_per_layer(w, cfg, int(round(T_mean)), False)
+    step_bytes = sum(decode_bytes_per_layer(w, cfg, int(round(T_mean)), fa) for fa in db.fa)
+
+    # ---------------- decode: end to end from pinned host buffers
+    q_h = db.q.cpu().pin_memory()
+    k_h = db.k_new.cpu().pin_memory()
+    v_h = db.v_new.cpu().pin_memory()
+    o_h = torch.empty(db.o.shape, dtype=db.o.dtype).pin_memory()
+    db.reset()
+    barrier(world)
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(args.steps):
+        db.q.copy_(q_h, non_blocking=True)
+        db.k_new.copy_(k_h, non_blocking=True)
+        db.v_new.copy_(v_h, non_blocking=True)
+        db.step()
+        o_h.copy_(db.o, non_blocking=True)
+    e2.record()
+    barrier(world)
+    t2 = max_over_ranks(s2.elapsed_time(e2), world)
+    e2e = {"value": world * w.batch * args.steps / (t2 / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": (q_h.numel() + k_h.numel() + v_h.numel()) * 2,
+           "d2h_bytes_per_step": o_h.numel() * 2,
+           "what": "per step: pinned-host q, k_new, v_new for all 32 layers copied in, the "
+                   "32-layer decode step, outputs of all layers copied out"}
+
+    # ---------------- routing mix: decode step time vs SA-layer fraction
+    mix = {}
+    n_mix_steps = max(5, min(20, args.steps))
+    perm_sa = db.sa_layers + [i for i in range(w.n_layers) if i not in db.sa_layers]
+    for frac in (0.0, 0.25, 0.5, 0.75, 1.0):
+        n_sa = int(round(frac * w.n_layers))
+        db.set_sa_layers(perm_sa[:n_sa])
+        db.reset()
+        db.step()
+        barrier(world)
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n_mix_steps):
+            db.step()
+        b.record()
+        barrier(world)
+        ms = max_over_ranks(a.elapsed_time(b), world) / n_mix_steps
+        mix[f"{int(frac * 100)}%"] = {"sa_layers": n_sa, "ms_per_step": ms,
+                                      "tokens_per_s": world * w.batch / (ms / 1e3)}
+    base = mix["0%"]["ms_per_step"]
+    for v in mix.values():
+        v["speedup_vs_all_fa"] = base / v["ms_per_step"]
+    db.set_sa_layers(db.sa_layers)
+    del db
+    torch.cuda.empty_cache()
+
+    # ---------------- prefill phase (Llama shape, 8192 tokens, router-chosen routes)
+    pb = PrefillBench(seed=99 + rank)
+    for _ in range(max(1, min(args.warmup, 3))):
+        pb.reset()
+        pb.step()
+    n_pf = max(3, min(10, args.steps))
+    pf_ms, fa_ev, rt_ev = [], [], []
+    barrier(world)
+    for _ in range(n_pf):
+        pb.reset()
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        pb.step(fa_events=fa_ev, router_events=rt_ev)
+        b.record()
+        pf_ms.append((a, b))
+    barrier(world)
+    pf_step = max_over_ranks(statistics.mean(elapsed_ms(pf_ms)), world)
+    fa_launch = statistics.mean(elapsed_ms(fa_ev))
+    flops_fa = prefill_flops_per_layer(pb.cfg, pb.w.seq, True)
+    flops_sa = prefill_flops_per_layer(pb.cfg, pb.w.seq, False)
+    n_fa = sum(pb.fa)
+    tflops = flops_fa / (fa_launch / 1e3) / 1e12
+    prefill = {
+        "workload": "llama3.1-8b-shape prefill, 1 x 8192 tokens, router 4096->256->32 "
+                    f"(seeded; {w.n_layers - n_fa} SA layers), SA sink 128 + window 2048",
+        "tokens_per_s": world * pb.w.batch * pb.w.seq / (pf_step / 1e3),
+        "ms_per_step": pf_step, "steps": n_pf, "sa_layers": pb.w.n_layers - n_fa,
+        "router_ms": statistics.mean(elapsed_ms(rt_ev)),
+        "algorithmic_tflops_per_step": (n_fa * flops_fa + (pb.w.n_layers - n_fa) * flops_sa) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128> (tcgen05), FA layers",
+                     "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tflops / peaks["bf16_tflops"],
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst)", "traffic": None,
+                     "launch_ms": fa_launch, "algorithmic_flops_per_launch": flops_fa},
+        "gpu_launches_per_step": pb.launches_per_step,
+    }
+    del pb
+    torch.cuda.empty_cache()
+
+    # ---------------- CPU baseline (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu:
+        t0 = time.perf_counter()
+        tok_s, per = cpu_baseline_decode_tok_s(w, len(sa_layers), n_seq=2)
+        cpu = {"value": tok_s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": "one decode token of 2 of the 16 sequences at 32768 context for one FA "
+                         "and one SA layer (fp64 oracle), scaled to 16 FA + 16 SA layers; "
+                         f"{time.perf_counter() - t0:.1f} s of CPU time"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": decode_config(w, cfg, sa_layers),
+        "roofline": roofline,
+        "decode_step": {"algorithmic_gb_per_step": step_bytes / 1e9,
+                        "step_gb_per_s": step_bytes / (ms_step / 1e3) / 1e9,
+                        "fa_layer_bytes": fa_bytes, "sa_layer_bytes": sa_bytes},
+        "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": w.n_layers * 4 * args.steps, "clocks": clocks,
+        "prefill": prefill, "routing_mix": mix,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["flux", "reference"], default="flux")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.warmup + args.steps > 256 - 1:
+        raise SystemExit("warm-up + steps must stay within the 256 decode steps of capacity")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_flux(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
