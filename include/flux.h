@@ -156,6 +156,35 @@ int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask
                 const int32_t* seq_len, int32_t batch, int32_t capacity, uint16_t* o,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the scratch array flux_decode_static keeps inside the library (32 MiB). */
+#define FLUX_DECODE_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * flux_decode_static -- flux_decode without a caller workspace.  The paper has no
+ * counterpart: this is a deployment convenience of this library.
+ *   Meant for callers that cannot allocate device memory or hand the library a
+ *   buffer: plugin hosts that give an op no scratch argument, real-time serving loops
+ *   that forbid allocation once they are running, and code that runs while some other
+ *   component owns the device allocator.
+ *   Same arguments and results as flux_decode, minus the workspace.  The split
+ *   partials go to a fixed FLUX_DECODE_STATIC_SCRATCH_BYTES array inside the library,
+ *   which every GPU that loads the library holds until the process exits; this call
+ *   allocates and frees nothing.
+ *   Limit: a call whose flux_decode_workspace_size(cfg, batch) exceeds
+ *   FLUX_DECODE_STATIC_SCRATCH_BYTES returns FLUX_ERR_WORKSPACE without launching
+ *   (the Llama-3.1-8B decode geometry fits up to batch 31).
+ *   The first call on a device looks up the array's device address (with that
+ *   device current) and caches it; make that first call before any stream capture.
+ *   All calls share the one array, so calls that can overlap on the GPU (different
+ *   streams, or devices sharing a context) race and corrupt each other's results;
+ *   serialise them.  The array keeps the last call's contents; nothing in it needs to
+ *   start at zero, because every record the combine pass reads is written first.
+ */
+int flux_decode_static(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                       const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                       const int32_t* seq_len, int32_t batch, int32_t capacity, uint16_t* o,
+                       void* stream);
+
 /*
  * flux_sa_block_ranges -- the SA key-block set of each query block, as the kernels
  * compute it (streaming pattern of Table 6).  For query block qb (queries

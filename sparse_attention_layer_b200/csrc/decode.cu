@@ -20,8 +20,18 @@
 //    to the caller's workspace; a combine kernel merges the splits and writes bf16.
 #include <math.h>
 
+#include <mutex>
+
+#include "../../include/flux.h"
 #include "flux_device.cuh"
 #include "flux_internal.h"
+
+// Scratch for flux_decode_static: the split partials that flux_decode keeps in the
+// caller's workspace, held instead in a fixed array inside the library image.  Every
+// GPU that loads the library reserves these bytes until the process exits.  In host
+// code this name is only a host-side stand-in: its device address comes from
+// cudaGetSymbolAddress (see static_scratch_address below).
+static __device__ __align__(256) unsigned char g_decode_static_scratch[FLUX_DECODE_STATIC_SCRATCH_BYTES];
 
 namespace flux {
 namespace {
@@ -480,6 +490,28 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_address[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device.  Looked up once per
+// device (with that device current) on its first use and cached.
+cudaError_t static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_address[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_decode_static_scratch);
+    if (err != cudaSuccess) return err;
+    g_static_address[dev] = p;
+  }
+  *out = g_static_address[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 
 size_t decode_workspace_bytes(const AttnGeom& g, int batch) {
@@ -527,6 +559,20 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
   FLUX_DECODE_CASE(64, 8)
 #undef FLUX_DECODE_CASE
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_static(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                                 const uint16_t* q, const uint16_t* k_cache,
+                                 const uint16_t* v_cache, const int32_t* seq_len, int batch,
+                                 int capacity, uint16_t* o, unsigned* status,
+                                 cudaStream_t stream) {
+  // The split kernel writes every partial record the combine kernel reads, so the
+  // scratch needs no clearing between calls.
+  void* scratch = nullptr;
+  const cudaError_t err = static_scratch_address(&scratch);
+  if (err != cudaSuccess) return err;
+  return launch_decode(g, layer, fa_mask, q, k_cache, v_cache, seq_len, batch, capacity, o,
+                       scratch, status, stream);
 }
 
 }  // namespace flux

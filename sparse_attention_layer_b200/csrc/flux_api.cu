@@ -220,6 +220,26 @@ int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask
                                                static_cast<cudaStream_t>(stream)));
 }
 
+int flux_decode_static(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                       const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                       const int32_t* seq_len, int32_t batch, int32_t capacity, uint16_t* o,
+                       void* stream) {
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!fa_mask || !q || !k_cache || !v_cache || !seq_len || !o) return FLUX_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= cfg->n_layers) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > flux::kDecMaxBatch || capacity < 1) return FLUX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return FLUX_ERR_INVALID_ARG;
+  const flux::AttnGeom g = flux::geom_of(cfg);
+  if (flux::decode_workspace_bytes(g, batch) > FLUX_DECODE_STATIC_SCRATCH_BYTES)
+    return FLUX_ERR_WORKSPACE;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  return flux::cuda_status(flux::launch_decode_static(g, layer, fa_mask, q, k_cache, v_cache,
+                                                      seq_len, batch, capacity, o, status,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
 int flux_sa_block_ranges(const flux_attn_cfg* cfg, int32_t n_qblocks, int32_t* ranges,
                          void* stream) {
   const int st = flux::validate_cfg(cfg);

@@ -24,6 +24,14 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
                           const int32_t* seq_len, int batch, int capacity, uint16_t* o,
                           void* workspace, unsigned* status, cudaStream_t stream);
 
+// Decode with the library's own file-scope scratch array instead of a caller
+// workspace (flux_decode_static).  Its size is FLUX_DECODE_STATIC_SCRATCH_BYTES.
+cudaError_t launch_decode_static(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                                 const uint16_t* q, const uint16_t* k_cache,
+                                 const uint16_t* v_cache, const int32_t* seq_len, int batch,
+                                 int capacity, uint16_t* o, unsigned* status,
+                                 cudaStream_t stream);
+
 // ----- KV append
 cudaError_t launch_kv_append(const AttnGeom& g, uint16_t* k_cache, uint16_t* v_cache,
                              int32_t* seq_len, int batch, int capacity, const uint16_t* k_new,

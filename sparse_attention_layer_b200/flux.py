@@ -33,8 +33,11 @@ FLUX_DEVICE_BAD_LENGTH = 0x4
 EXPORTED = (
     "flux_mask_words", "flux_route", "flux_kv_append", "flux_prefill",
     "flux_decode_workspace_size", "flux_decode", "flux_sa_block_ranges",
-    "flux_get_device_status", "flux_status_string", "flux_version",
+    "flux_get_device_status", "flux_status_string", "flux_version", "flux_decode_static",
 )
+
+# bytes of the scratch array flux_decode_static keeps inside the library
+FLUX_DECODE_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class FluxError(RuntimeError):
@@ -115,6 +118,9 @@ def lib() -> ctypes.CDLL:
         L.flux_decode.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32, i32,
                                   vp, vp, sz, vp]
         L.flux_decode.restype = ctypes.c_int
+        L.flux_decode_static.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32,
+                                         i32, vp, vp]
+        L.flux_decode_static.restype = ctypes.c_int
         L.flux_sa_block_ranges.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp]
         L.flux_sa_block_ranges.restype = ctypes.c_int
         _lib = L
@@ -248,6 +254,25 @@ def flux_decode(cfg: AttnCfg, layer: int, fa_mask, q, k_cache, v_cache, seq_len,
         _ptr(o, "o", torch.bfloat16, (batch, hq, d)),
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check("flux_decode", st)
+
+
+def flux_decode_static(cfg: AttnCfg, layer: int, fa_mask, q, k_cache, v_cache, seq_len, o,
+                       stream=None) -> None:
+    """flux_decode without a workspace argument, for callers that cannot allocate
+    device memory: the library's own fixed scratch array (FLUX_DECODE_STATIC_SCRATCH_BYTES)
+    holds the split partials.  Calls that overlap on the GPU share that array and race;
+    the first call on a device should come before any stream capture."""
+    batch, hq, d = q.shape
+    cap = k_cache.shape[2]
+    c = cfg.c()
+    st = lib().flux_decode_static(
+        ctypes.byref(c), int(layer), _ptr(fa_mask, "fa_mask", torch.int32, (batch, cfg.mask_words)),
+        _ptr(q, "q", torch.bfloat16), _ptr(k_cache, "k_cache", torch.bfloat16,
+                                           (batch, cfg.n_kv_heads, cap, d)),
+        _ptr(v_cache, "v_cache", torch.bfloat16, (batch, cfg.n_kv_heads, cap, d)),
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, cap,
+        _ptr(o, "o", torch.bfloat16, (batch, hq, d)), _stream(stream))
+    _check("flux_decode_static", st)
 
 
 def flux_sa_block_ranges(cfg: AttnCfg, n_qblocks: int, ranges, stream=None) -> None:
