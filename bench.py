@@ -105,6 +105,26 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def measured_traffic(kernel: str, units: float):
+    """DRAM bytes per launch of `kernel` scaled from the committed ncu capture in
+    profiles/traffic.txt to `units` (sequences for decode, prompts for prefill); None
+    when the capture is missing or the kernel's sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as f:
+            kv = dict(line.split(" = ", 1) for line in f.read().splitlines()
+                      if " = " in line and not line.startswith("#"))
+        for item in kv[f"{kernel}.sources"].split():
+            rel, digest = item.split(":")
+            with open(os.path.join(ROOT, "sparse_attention_layer_b200", rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
+                    return None
+        return float(kv[f"{kernel}.bytes"]) / float(kv[f"{kernel}.units"]) * units
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def dist_setup(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -427,7 +447,9 @@ def run_flux(args, world, rank, local):
     roofline = {"bound": "hbm", "kernel": "flux_decode (split-KV + combine), FA layers",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_kind": f"{peak_kind} hbm_gbs",
-                "traffic": None, "launch_ms": statistics.mean(fa_ms),
+                "traffic": measured_traffic("decode_split", w.batch),
+                "traffic_note": "ncu dram bytes of a 4-sequence capture scaled to 16",
+                "launch_ms": statistics.mean(fa_ms),
                 "algorithmic_bytes_per_launch": fa_bytes}
     sa_bytes = decode_bytes_per_layer(w, cfg, int(round(T_mean)), False)
     step_bytes = sum(decode_bytes_per_layer(w, cfg, int(round(T_mean)), fa) for fa in db.fa)
@@ -515,7 +537,8 @@ def run_flux(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128> (tcgen05), FA layers",
                      "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tflops / peaks["bf16_tflops"],
-                     "peak_kind": f"{peak_kind} bf16_tflops (burst)", "traffic": None,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst)",
+                     "traffic": measured_traffic("prefill", pb.w.batch),
                      "launch_ms": fa_launch, "algorithmic_flops_per_launch": flops_fa},
         "gpu_launches_per_step": pb.launches_per_step,
     }
