@@ -9,12 +9,14 @@
 //    >= 128 keys; a persistent grid (one CTA per SM) walks the (sequence, KV head,
 //    split) items round-robin, so SA layers launch no idle CTAs;
 //  * one producer lane streams each split's K and V rows -- contiguous in the
-//    [B][Hkv][cap][d] cache -- into a 4-stage shared-memory ring with 1-D bulk copies
-//    (cp.async.bulk, no cluster), completing on mbarriers;
-//  * 8 consumer warps read the stage with 128-bit shared loads: 8 lanes cover one
-//    key row (16 B each), 4 rows per warp instruction, all G = Hq/Hkv query heads of
-//    the group at once; the q.k partial sums are reduced across the 8 lanes with a
-//    transposing butterfly (G values in log2(G)+... shuffles instead of G*3);
+//    [B][Hkv][cap][d] cache -- into a 3-stage ring of 128-key stages with 1-D bulk
+//    copies (cp.async.bulk, no cluster), completing on mbarriers; the group's query
+//    rows ride along with the first stage of every split;
+//  * 8 consumer warps (16 keys each per stage) read the stage with 128-bit shared
+//    loads: 8 lanes cover one key row (16 B each), 4 rows per warp instruction, all
+//    G = Hq/Hkv query heads of the group at once, with packed fp32x2 FMAs; the q.k
+//    partial sums are reduced across the 8 lanes with a transposing butterfly (each
+//    level hands half of the remaining head sums to the partner lane);
 //  * online softmax in the log2 domain per head; P.V accumulates in fp32 registers;
 //  * each item writes (running max, running sum, unnormalised accumulator) per head
 //    to the caller's workspace; a combine kernel merges the splits and writes bf16.
@@ -36,12 +38,13 @@ static __device__ __align__(256) unsigned char g_decode_static_scratch[FLUX_DECO
 namespace flux {
 namespace {
 
-constexpr int kStageKeys = 64;
-constexpr int kStages = 4;
+constexpr int kStageKeys = 128;
+constexpr int kMaxStages = 3;
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kKeysPerWarp = kStageKeys / kConsumerWarps;  // 8 keys per warp per stage
+constexpr int kKeysPerWarp = kStageKeys / kConsumerWarps;  // 16 keys per warp per stage
 constexpr int kPasses = kKeysPerWarp / 4;                  // 4 keys per warp instruction
+static_assert(kPasses == 4, "the tile maximum below is written for 4 passes");
 
 struct DecodeArgs {
   const uint32_t* fa_mask;
@@ -52,6 +55,7 @@ struct DecodeArgs {
   const int32_t* seq_len;
   int batch, capacity, hkv, block, sink, window;
   float scale_log2;  // log2(e) / sqrt(d)
+  int min_splits;    // splits per (sequence, KV head) that give every SM 2 items
   float* ws_acc;     // [B][Hkv][kDecMaxSplits][G][D]
   float2* ws_ml;     // [B][Hkv][kDecMaxSplits][G] = (max, sum)
   uint16_t* o;
@@ -73,8 +77,14 @@ __device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
   p.len0 = r.hi0 - r.lo0;
   p.lo1 = r.lo1;
   p.n_vis = p.len0 + (r.hi1 - r.lo1);
-  const int s = (p.n_vis + kDecMinChunk - 1) / kDecMinChunk;
-  p.n_split = s < kDecMaxSplits ? s : kDecMaxSplits;
+  // splits: enough items for every SM (min_splits), at most kDecMaxChunk keys each
+  // when the split budget allows, never fewer than kDecMinChunk keys.
+  const int by_min = (p.n_vis + kDecMinChunk - 1) / kDecMinChunk;
+  const int by_max = (p.n_vis + kDecMaxChunk - 1) / kDecMaxChunk;
+  int s = by_max > a.min_splits ? by_max : a.min_splits;
+  if (s > by_min) s = by_min;
+  if (s > kDecMaxSplits) s = kDecMaxSplits;
+  p.n_split = s;
   p.chunk = (p.n_vis + p.n_split - 1) / p.n_split;
   return p;
 }
@@ -193,12 +203,44 @@ __device__ __forceinline__ float group_reduce(float (&v)[G], int lane) {
   }
 }
 
-template <int D, int G>
-struct DecodeSmem {
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of a float pair.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// bf16 pair (one 32-bit word) -> the two values as an fp32 pair, exactly.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+template <int D, int G, int S>
+struct DecodeSmemLayout {
+  static constexpr int kStages = S;
   static constexpr size_t kv_stage = size_t(kStageKeys) * D;  // elements per stage
+  static constexpr size_t q_slot = size_t(G) * D;              // elements per q slot
   static constexpr size_t off_k = 0;
   static constexpr size_t off_v = off_k + kStages * kv_stage * 2;
-  static constexpr size_t off_p = off_v + kStages * kv_stage * 2;               // float
+  static constexpr size_t off_q = off_v + kStages * kv_stage * 2;
+  static constexpr size_t off_p = off_q + kStages * q_slot * 2;                  // float
   static constexpr size_t off_acc = off_p + kConsumerWarps * kKeysPerWarp * G * 4;
   static constexpr size_t off_m = off_acc + size_t(kConsumerWarps) * G * D * 4;
   static constexpr size_t off_l = off_m + kConsumerWarps * G * 4;
@@ -207,14 +249,22 @@ struct DecodeSmem {
   static size_t bytes(int batch) { return off_prefix + size_t(batch + 1) * 4; }
 };
 
+// As many stages (up to 3) as fit in 220 KB of shared memory with a 1024-sequence
+// length table: 3 for every geometry except d = 128 with 8 query heads per KV head.
+template <int D, int G>
+using DecodeSmem = DecodeSmemLayout<
+    D, G, (DecodeSmemLayout<D, G, kMaxStages>::off_prefix + 4100 <= 220 * 1024) ? kMaxStages : 2>;
+
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeArgs a) {
   using L = DecodeSmem<D, G>;
+  constexpr int kStages = L::kStages;
   constexpr int NCH = D / 64;          // 16-byte chunks of a row per lane
   constexpr int GB = (G == 1) ? 0 : (G == 2) ? 1 : (G == 4) ? 2 : 3;
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* sK = reinterpret_cast<uint16_t*>(smem + L::off_k);
   uint16_t* sV = reinterpret_cast<uint16_t*>(smem + L::off_v);
+  uint16_t* sQ = reinterpret_cast<uint16_t*>(smem + L::off_q);
   float* sP = reinterpret_cast<float*>(smem + L::off_p);
   float* sAcc = reinterpret_cast<float*>(smem + L::off_acc);
   float* sM = reinterpret_cast<float*>(smem + L::off_m);
@@ -268,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const Item it = item_at(a, prefix, idx);
         const size_t head_off = (size_t(it.b) * a.hkv + it.kvh) * a.capacity * row_elems;
+        const uint16_t* qsrc = a.q + (size_t(it.b) * a.hkv * G + size_t(it.kvh) * G) * D;
         const int ns = item_stages(it);
         for (int k = 0; k < ns; ++k, ++g) {
           int pos, n;
@@ -276,7 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
           const uint32_t ph = (g / kStages) & 1;
           if (!mbar_wait(empty0 + 8 * st, ph ^ 1, a.status)) { ok = false; break; }
           const uint32_t bytes = uint32_t(n) * D * 2;
-          mbar_arrive_expect_tx(full0 + 8 * st, 2 * bytes);
+          const uint32_t qbytes = (k == 0) ? uint32_t(G * D * 2) : 0u;
+          mbar_arrive_expect_tx(full0 + 8 * st, 2 * bytes + qbytes);
+          if (k == 0) bulk_g2s(smem_addr(sQ + st * L::q_slot), qsrc, qbytes, full0 + 8 * st, pol);
           bulk_g2s(smem_addr(sK + st * L::kv_stage), a.k + head_off + size_t(pos) * row_elems,
                    bytes, full0 + 8 * st, pol);
           bulk_g2s(smem_addr(sV + st * L::kv_stage), a.v + head_off + size_t(pos) * row_elems,
@@ -302,25 +355,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
   bool ok = true;
   for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
     const Item it = item_at(a, prefix, idx);
-    float qf[G][8 * NCH];
-    {
-      const uint16_t* qp = a.q + (size_t(it.b) * a.hkv * G + size_t(it.kvh) * G) * D;
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qp + h * D + ch * 64 + c * 8));
-          float f[8];
-          bf16x8_to_float(raw, f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) qf[h][ch * 8 + e] = f[e] * a.scale_log2;
-        }
-    }
-    float acc[G][8 * NCH];
+    uint64_t q2[G][4 * NCH];   // pre-scaled query pairs of this lane's 8*NCH dims
+    uint64_t acc[G][4 * NCH];  // P.V pairs of this lane's dims
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8 * NCH; ++e) acc[h][e] = 0.f;
+      for (int i = 0; i < 4 * NCH; ++i) acc[h][i] = 0ull;
     float m_run = -INFINITY, l_run = 0.f;
 
     const int ns = item_stages(it);
@@ -330,6 +370,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       const int st = g % kStages;
       const uint32_t ph = (g / kStages) & 1;
       if (!mbar_wait(full0 + 8 * st, ph, a.status)) { ok = false; break; }
+      if (k == 0) {
+        const uint64_t sc = f2_pack(a.scale_log2, a.scale_log2);
+        const uint16_t* qs = sQ + st * L::q_slot;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch) {
+            const uint4 raw = lds128(qs + h * D + ch * 64 + c * 8);
+            q2[h][ch * 4 + 0] = f2_mul(bf16x2_to_f2(raw.x), sc);
+            q2[h][ch * 4 + 1] = f2_mul(bf16x2_to_f2(raw.y), sc);
+            q2[h][ch * 4 + 2] = f2_mul(bf16x2_to_f2(raw.z), sc);
+            q2[h][ch * 4 + 3] = f2_mul(bf16x2_to_f2(raw.w), sc);
+          }
+      }
       const uint16_t* Ks = sK + st * L::kv_stage;
       const uint16_t* Vs = sV + st * L::kv_stage;
 
@@ -337,25 +391,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
 #pragma unroll
       for (int p = 0; p < kPasses; ++p) {
         const int key = warp * kKeysPerWarp + p * 4 + key_sub;
-        float dot[G];
+        uint64_t dot2[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) dot[h] = 0.f;
+        for (int h = 0; h < G; ++h) dot2[h] = 0ull;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
           const uint4 raw = lds128(Ks + key * D + ch * 64 + c * 8);
-          float kf[8];
-          bf16x8_to_float(raw, kf);
+          const uint64_t k0 = bf16x2_to_f2(raw.x), k1 = bf16x2_to_f2(raw.y);
+          const uint64_t k2 = bf16x2_to_f2(raw.z), k3 = bf16x2_to_f2(raw.w);
 #pragma unroll
-          for (int h = 0; h < G; ++h)
+          for (int h = 0; h < G; ++h) {
+            dot2[h] = f2_fma(q2[h][ch * 4 + 0], k0, dot2[h]);
+            dot2[h] = f2_fma(q2[h][ch * 4 + 1], k1, dot2[h]);
+            dot2[h] = f2_fma(q2[h][ch * 4 + 2], k2, dot2[h]);
+            dot2[h] = f2_fma(q2[h][ch * 4 + 3], k3, dot2[h]);
+          }
+        }
+        float dot[G];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dot[h] = fmaf(qf[h][ch * 8 + e], kf[e], dot[h]);
+        for (int h = 0; h < G; ++h) {
+          float lo, hi;
+          f2_unpack(dot2[h], lo, hi);
+          dot[h] = lo + hi;
         }
         const float r = group_reduce<G>(dot, lane);
         s[p] = (key < n) ? r : -INFINITY;
       }
-      float mt = s[0];
-#pragma unroll
-      for (int p = 1; p < kPasses; ++p) mt = fmaxf(mt, s[p]);
+      float mt = fmax3(s[0], s[1], s[2]);
+      mt = fmaxf(mt, s[3]);
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
       const float m_new = fmaxf(m_run, mt);
@@ -365,8 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float ah = __shfl_sync(0xffffffffu, alpha, group_lane0 | (h << (3 - GB)));
+          const uint64_t ah2 = f2_pack(ah, ah);
 #pragma unroll
-          for (int e = 0; e < 8 * NCH; ++e) acc[h][e] *= ah;
+          for (int i = 0; i < 4 * NCH; ++i) acc[h][i] = f2_mul(acc[h][i], ah2);
         }
         m_run = m_new;
       }
@@ -383,18 +447,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       for (int p = 0; p < kPasses; ++p) {
         const int key = warp * kKeysPerWarp + p * 4 + key_sub;
         if (key < n) {
-          float pw[G];
+          uint64_t pw2[G];
 #pragma unroll
-          for (int h = 0; h < G; ++h) pw[h] = Pw[(p * 4 + key_sub) * G + h];
+          for (int h = 0; h < G; ++h) {
+            const float pw = Pw[(p * 4 + key_sub) * G + h];
+            pw2[h] = f2_pack(pw, pw);
+          }
 #pragma unroll
           for (int ch = 0; ch < NCH; ++ch) {
             const uint4 raw = lds128(Vs + key * D + ch * 64 + c * 8);
-            float vf[8];
-            bf16x8_to_float(raw, vf);
+            const uint64_t v0 = bf16x2_to_f2(raw.x), v1 = bf16x2_to_f2(raw.y);
+            const uint64_t v2 = bf16x2_to_f2(raw.z), v3 = bf16x2_to_f2(raw.w);
 #pragma unroll
-            for (int h = 0; h < G; ++h)
-#pragma unroll
-              for (int e = 0; e < 8; ++e) acc[h][ch * 8 + e] = fmaf(pw[h], vf[e], acc[h][ch * 8 + e]);
+            for (int h = 0; h < G; ++h) {
+              acc[h][ch * 4 + 0] = f2_fma(pw2[h], v0, acc[h][ch * 4 + 0]);
+              acc[h][ch * 4 + 1] = f2_fma(pw2[h], v1, acc[h][ch * 4 + 1]);
+              acc[h][ch * 4 + 2] = f2_fma(pw2[h], v2, acc[h][ch * 4 + 2]);
+              acc[h][ch * 4 + 3] = f2_fma(pw2[h], v3, acc[h][ch * 4 + 3]);
+            }
           }
         }
       }
@@ -404,25 +474,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
     if (!ok) break;
 
     // reduce the 4 row groups of the warp, then the 8 warps through shared memory
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8 * NCH; ++e) {
-        acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 8);
-        acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 16);
+      for (int i = 0; i < 4 * NCH; ++i) {
+        float lo, hi;
+        f2_unpack(acc[h][i], lo, hi);
+        lo += __shfl_xor_sync(0xffffffffu, lo, 8);
+        hi += __shfl_xor_sync(0xffffffffu, hi, 8);
+        lo += __shfl_xor_sync(0xffffffffu, lo, 16);
+        hi += __shfl_xor_sync(0xffffffffu, hi, 16);
+        acc[h][i] = f2_pack(lo, hi);
       }
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
     if (key_sub == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
+          float f[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) f2_unpack(acc[h][ch * 4 + i], f[2 * i], f[2 * i + 1]);
           float4* dst = reinterpret_cast<float4*>(sAcc + (warp * G + h) * D + ch * 64 + c * 8);
-          dst[0] = make_float4(acc[h][ch * 8 + 0], acc[h][ch * 8 + 1], acc[h][ch * 8 + 2],
-                               acc[h][ch * 8 + 3]);
-          dst[1] = make_float4(acc[h][ch * 8 + 4], acc[h][ch * 8 + 5], acc[h][ch * 8 + 6],
-                               acc[h][ch * 8 + 7]);
+          dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+          dst[1] = make_float4(f[4], f[5], f[6], f[7]);
         }
       if (owner) {
         sM[warp * G + hl] = m_run;
@@ -451,26 +527,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
   }
 }
 
+// Merge the split partials of one (sequence, KV head): weights 2^(m_s - M) / L are
+// computed once per (split, head) in shared memory, then the partial accumulators are
+// read coalesced along d.
 template <int D, int G>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int kvh = h / G, gi = h % G;
+__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
+  __shared__ float wgt[kDecMaxSplits][G];
+  const int kvh = blockIdx.x, b = blockIdx.y;
   const Plan p = make_plan(a, b);
-  uint16_t* out = a.o + (size_t(b) * a.hkv * G + h) * D;
   const size_t rec0 = (size_t(b) * a.hkv + kvh) * kDecMaxSplits;
-  float M = -INFINITY;
-  for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, a.ws_ml[(rec0 + s) * G + gi].x);
-  for (int e = threadIdx.x; e < D; e += blockDim.x) {
-    float lv = 0.f, av = 0.f;
-    for (int s = 0; s < p.n_split; ++s) {
-      const float2 ml = a.ws_ml[(rec0 + s) * G + gi];
-      const float f = fast_exp2(ml.x - M);
-      lv = fmaf(f, ml.y, lv);
-      av = fmaf(f, a.ws_acc[((rec0 + s) * G + gi) * D + e], av);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (warp < G) {
+    // one warp per query head of the group: splits spread over the lanes
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    if (lane < p.n_split) {
+      const float2 ml = a.ws_ml[(rec0 + lane) * G + warp];
+      m0 = ml.x; l0 = ml.y;
     }
-    const float r = (p.n_split > 0) ? av / lv : 0.f;
-    const __nv_bfloat16 hb = __float2bfloat16_rn(r);
-    out[e] = *reinterpret_cast<const uint16_t*>(&hb);
+    if (lane + 32 < p.n_split) {
+      const float2 ml = a.ws_ml[(rec0 + lane + 32) * G + warp];
+      m1 = ml.x; l1 = ml.y;
+    }
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float f0 = (lane < p.n_split) ? fast_exp2(m0 - M) : 0.f;
+    const float f1 = (lane + 32 < p.n_split) ? fast_exp2(m1 - M) : 0.f;
+    float lv = f0 * l0 + f1 * l1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, off);
+    const float inv = (lv > 0.f) ? 1.f / lv : 0.f;
+    if (lane < p.n_split) wgt[lane][warp] = f0 * inv;
+    if (lane + 32 < p.n_split) wgt[lane + 32][warp] = f1 * inv;
+  }
+  __syncthreads();
+  uint16_t* out = a.o + (size_t(b) * a.hkv * G + size_t(kvh) * G) * D;
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int gi = i / D, e = i % D;
+    const float* src = a.ws_acc + (rec0 * G + gi) * D + e;
+    float av0 = 0.f, av1 = 0.f, av2 = 0.f, av3 = 0.f;
+    int s = 0;
+    for (; s + 4 <= p.n_split; s += 4) {
+      av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
+      av1 = fmaf(wgt[s + 1][gi], src[size_t(s + 1) * G * D], av1);
+      av2 = fmaf(wgt[s + 2][gi], src[size_t(s + 2) * G * D], av2);
+      av3 = fmaf(wgt[s + 3][gi], src[size_t(s + 3) * G * D], av3);
+    }
+    for (; s < p.n_split; ++s) av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
+    const __nv_bfloat16 hb = __float2bfloat16_rn((av0 + av1) + (av2 + av3));
+    out[gi * D + e] = *reinterpret_cast<const uint16_t*>(&hb);
   }
 }
 
@@ -478,15 +584,25 @@ template <int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   using L = DecodeSmem<D, G>;
   const size_t smem = L::bytes(a.batch);
-  cudaError_t err = cudaFuncSetAttribute(decode_split_kernel<D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  // the attribute is per device; set it (to the largest size any batch needs) once
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    err = cudaFuncSetAttribute(decode_split_kernel<D, G>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(L::bytes(kDecMaxBatch)));
+    if (err != cudaSuccess) return err;
+    attr_set[dev] = true;
+  }
   const int max_items = a.batch * a.hkv * kDecMaxSplits;
   const int grid = min(max_items, device_sm_count());
   decode_split_kernel<D, G><<<grid, kThreads, smem, stream>>>(a);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  decode_combine_kernel<D, G><<<dim3(a.hkv * G, a.batch), 128, 0, stream>>>(a);
+  decode_combine_kernel<D, G><<<dim3(a.hkv, a.batch), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -541,6 +657,10 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
   a.sink = g.sink;
   a.window = g.window;
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(g.head_dim)));
+  {
+    const int pairs = batch * g.hkv;
+    a.min_splits = (2 * device_sm_count() + pairs - 1) / pairs;
+  }
   const size_t recs = size_t(batch) * g.hkv * kDecMaxSplits * G;
   a.ws_acc = static_cast<float*>(workspace);
   a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) +
