@@ -4,26 +4,35 @@
 // window of blocks) visits only the sink tiles and the window tiles.  The route is
 // read on the device from the layer's bit of the router's mask (Figure 2).
 //
-// One CTA computes one 128-query tile of one query head.  Roles (192 threads):
-//   warps 0-3  softmax: thread i owns query row i; it reads its row of S = Q K^T from
-//              tensor memory (tcgen05.ld), masks boundary tiles, runs the online
-//              softmax in registers (log2 domain, a stale row maximum that is only
-//              raised when the new maximum exceeds it by more than 2^8, in which case
-//              the O row in tensor memory is rescaled), writes P as bf16 into shared
-//              memory in the 128-byte-swizzled K-major layout the MMA reads, and at
-//              the end normalises O and stores it.
-//   warp 4     TMA producer: the Q tile once, then K and V tiles into a 2-stage ring
-//              (cp.async.bulk.tensor, 128-byte swizzle, no cluster, no multicast).
-//   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two S buffers in
-//              tensor memory, then O += P_j V_j into the O accumulator; completion is
-//              signalled with tcgen05.commit on mbarriers.  The warp also allocates
-//              and frees the 512 tensor-memory columns (S0 | S1 | O).
+// One CTA computes one 128-query tile of one query head.  Roles (352 threads):
+//   warps 0-7  softmax, two warpgroups: warpgroup h (h = 0, 1) owns columns
+//              [64h, 64h + 64) of each 128-key tile for all 128 query rows (thread =
+//              one row in one half).  It reads its half of S = Q K^T from tensor
+//              memory (tcgen05.ld), masks boundary tiles, swaps half-row maxima with
+//              the other warpgroup through shared memory, runs the online softmax in
+//              registers (log2 domain; a stale row maximum raised only when the new
+//              maximum exceeds it by more than 2^8, and then O is rescaled in tensor
+//              memory), and writes P as bf16 back into tensor memory over its own S
+//              columns, where the P.V MMA reads it as its A operand.  At the end it
+//              normalises its half of the O row and stores it.
+//   warps 8-9  TMA producers (cp.async.bulk.tensor, 128-byte swizzle, no cluster, no
+//              multicast): warp 8 the Q tile once and K tiles into a 3-stage ring that
+//              is released as soon as each tile's S MMAs complete; warp 9 V tiles into
+//              a 2-stage ring released by the P.V MMAs.
+//   warp 10    MMA issuer (one thread): S_j = Q K_j^T (A, B from shared memory) into
+//              one of three S buffers in tensor memory, then O += P_j V_j with P_j
+//              read from tensor memory and V_j an MN-major shared-memory operand;
+//              completion is signalled with tcgen05.commit on mbarriers.  The warp
+//              also allocates and frees the 512 tensor-memory columns
+//              (S0 | S1 | S2 | O).
 // S_{j+1} is issued before P_j V_j, so the tensor cores compute the next scores while
-// the softmax warps work on the current ones.
+// the softmax warps work on the current ones; with three S buffers, the buffer S_{j+1}
+// lands in last held P_{j-2}, whose P.V MMA was issued two MMA groups earlier.
 //
 // Every mbarrier wait is bounded: on time-out the thread records FLUX_DEVICE_TIMEOUT
 // and leaves its loop; all roles meet at the final barrier, the producer first waits
-// for its copies in flight, and the tensor memory is always freed.
+// for its copies in flight, the MMA thread for its MMAs, and the tensor memory is
+// always freed.
 #include <cuda.h>
 #include <math.h>
 
@@ -35,11 +44,16 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (MMA M)
 constexpr int BN = 128;  // keys per KV tile (MMA N of Q K^T, MMA K of P V)
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kKStages = 3;  // K tiles: released as soon as their S MMA completes
+constexpr int kVStages = 2;  // V tiles: released when their P.V MMA completes
+constexpr int kSoftmaxThreads = 256;
+constexpr int kKProducerWarp = 8;
+constexpr int kVProducerWarp = 9;
+constexpr int kMmaWarp = 10;
+constexpr int kThreads = 352;
+constexpr int kSBufs = 3;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 384;           // O accumulator columns [384, 384 + D)
 constexpr uint32_t kSubBytes = 128 * 128;  // one 64-column swizzled sub-tile of 128 rows
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -49,11 +63,13 @@ struct Smem {
   static constexpr uint32_t tile = NCH * kSubBytes;  // Q tile or one K / V tile
   static constexpr uint32_t off_q = 0;
   static constexpr uint32_t off_k = off_q + tile;
-  static constexpr uint32_t off_v = off_k + kStages * tile;
-  static constexpr uint32_t off_p = off_v + kStages * tile;
-  static constexpr uint32_t off_bar = off_p + 2 * kSubBytes;
-  // q_full | k_full[S] | v_full[S] | kv_empty[S] | s_full[2] | p_full | o_done | mma_idle
-  static constexpr int n_bars = 1 + 3 * kStages + 2 + 3;
+  static constexpr uint32_t off_v = off_k + kKStages * tile;
+  static constexpr uint32_t off_red = off_v + kVStages * tile;  // float [2][2][128] maxima
+  static constexpr uint32_t off_lsum = off_red + 2 * 2 * 128 * 4;  // float [2][128]
+  static constexpr uint32_t off_bar = off_lsum + 2 * 128 * 4;
+  // q_full | k_full[3] | k_empty[3] | v_full[2] | v_empty[2] | s_full[3] | p_full |
+  // o_done | o_final | mma_idle
+  static constexpr int n_bars = 1 + 2 * kKStages + 2 * kVStages + kSBufs + 4;
   static constexpr uint32_t off_tmem = off_bar + n_bars * 8;
   static constexpr uint32_t used = off_tmem + 16;
   // 1 KB slack to align the base; at least 116 KB so that a second CTA (which would
@@ -132,6 +148,24 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Same with the A operand (M x 16 bf16, one row per lane, pairs packed per column)
+// read from tensor memory.
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -252,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
   using L = Smem<D>;
   constexpr int NCH = L::NCH;
+  constexpr int DH = D / 2;  // O columns per softmax warpgroup
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -260,16 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = base + L::off_q;
   const uint32_t sK = base + L::off_k;
   const uint32_t sV = base + L::off_v;
-  const uint32_t sP = base + L::off_p;
+  float* red = reinterpret_cast<float*>(smem + L::off_red);
+  float* lsum = reinterpret_cast<float*>(smem + L::off_lsum);
   const uint32_t bar0 = base + L::off_bar;
   const uint32_t bar_q = bar0;
-  const uint32_t bar_kfull = bar0 + 8;                      // + 8 * stage
-  const uint32_t bar_vfull = bar0 + 8 * (1 + kStages);
-  const uint32_t bar_empty = bar0 + 8 * (1 + 2 * kStages);
-  const uint32_t bar_sfull = bar0 + 8 * (1 + 3 * kStages);  // + 8 * buffer
-  const uint32_t bar_pfull = bar0 + 8 * (3 + 3 * kStages);
-  const uint32_t bar_odone = bar0 + 8 * (4 + 3 * kStages);
-  const uint32_t bar_idle = bar0 + 8 * (5 + 3 * kStages);
+  const uint32_t bar_kfull = bar0 + 8;                        // + 8 * K stage
+  const uint32_t bar_kempty = bar_kfull + 8 * kKStages;
+  const uint32_t bar_vfull = bar_kempty + 8 * kKStages;       // + 8 * V stage
+  const uint32_t bar_vempty = bar_vfull + 8 * kVStages;
+  const uint32_t bar_sfull = bar_vempty + 8 * kVStages;       // + 8 * S buffer
+  const uint32_t bar_pfull = bar_sfull + 8 * kSBufs;
+  const uint32_t bar_odone = bar_pfull + 8;
+  const uint32_t bar_ofinal = bar_pfull + 16;
+  const uint32_t bar_idle = bar_pfull + 24;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_tmem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -291,15 +329,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar_kfull + 8 * s, 1);
-      mbar_init(bar_vfull + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_kempty + 8 * s, 1);
     }
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_sfull + 8, 1);
-    mbar_init(bar_pfull, 4);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar_vfull + 8 * s, 1);
+      mbar_init(bar_vempty + 8 * s, 1);
+    }
+    for (int s = 0; s < kSBufs; ++s) mbar_init(bar_sfull + 8 * s, 1);
+    mbar_init(bar_pfull, kSoftmaxThreads / 32);
     mbar_init(bar_odone, 1);
+    mbar_init(bar_ofinal, 1);
     mbar_init(bar_idle, 1);
     fence_barrier_init();
   }
@@ -314,43 +355,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_S0 = tmem;         // columns [0, 128)
-  const uint32_t tmem_O = tmem + 256;    // columns [256, 256 + D)
 
-  if (warp == kProducerWarp) {
-    // ---------------------------------------------------------------- TMA producer
-    int issued = 0;
+  if (warp == kKProducerWarp || warp == kVProducerWarp) {
+    // ---------------------------------------------------------------- TMA producers
+    // warp 8 loads Q and the K ring, warp 9 the V ring; each waits only on its own
+    // ring's release barriers, so K runs up to three tiles ahead of the MMAs.
     if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(bar_q, L::tile);
-      for (int c = 0; c < NCH; ++c)
-        tma_load_4d(sQ + c * kSubBytes, &tmQ, c * 64, h, row0, b, bar_q);
+      const bool is_k = (warp == kKProducerWarp);
+      const int n_st = is_k ? kKStages : kVStages;
+      const uint32_t full = is_k ? bar_kfull : bar_vfull;
+      const uint32_t empty = is_k ? bar_kempty : bar_vempty;
+      const uint32_t ring = is_k ? sK : sV;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      prefetch_tmap(map);
+      if (is_k) {
+        prefetch_tmap(&tmQ);
+        mbar_arrive_expect_tx(bar_q, L::tile);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_4d(sQ + c * kSubBytes, &tmQ, c * 64, h, row0, b, bar_q);
+      }
       const int kv_row = b * a.hkv + kvh;
+      int issued = 0;
       for (int j = 0; j < plan.n_tiles; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (!mbar_wait(bar_empty + 8 * st, ph ^ 1, a.status)) break;
+        const int st = j % n_st;
+        const uint32_t ph = (j / n_st) & 1;
+        if (!mbar_wait(empty + 8 * st, ph ^ 1, a.status)) break;
         const int k0 = tile_key0(plan, j);
-        mbar_arrive_expect_tx(bar_kfull + 8 * st, L::tile);
+        mbar_arrive_expect_tx(full + 8 * st, L::tile);
         for (int c = 0; c < NCH; ++c)
-          tma_load_3d(sK + st * L::tile + c * kSubBytes, &tmK, c * 64, k0, kv_row,
-                      bar_kfull + 8 * st);
-        mbar_arrive_expect_tx(bar_vfull + 8 * st, L::tile);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_3d(sV + st * L::tile + c * kSubBytes, &tmV, c * 64, k0, kv_row,
-                      bar_vfull + 8 * st);
+          tma_load_3d(ring + st * L::tile + c * kSubBytes, map, c * 64, k0, kv_row, full + 8 * st);
         ++issued;
       }
       // wait for the copies in flight before the CTA may exit
-      mbar_wait(bar_q, 0, a.status);
-      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        mbar_wait(bar_kfull + 8 * st, ph, a.status);
-        mbar_wait(bar_vfull + 8 * st, ph, a.status);
-      }
+      if (is_k) mbar_wait(bar_q, 0, a.status);
+      for (int j = (issued > n_st ? issued - n_st : 0); j < issued; ++j)
+        mbar_wait(full + 8 * (j % n_st), (j / n_st) & 1, a.status);
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
@@ -358,7 +397,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = make_idesc(BM, BN, false, false);
       constexpr uint32_t idesc_o = make_idesc(BM, D, false, true);
       bool ok = mbar_wait(bar_q, 0, a.status);
-      // S_0
       if (ok && plan.n_tiles > 0) {
         ok = mbar_wait(bar_kfull, 0, a.status);
         if (ok) {
@@ -366,41 +404,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
-            mma_bf16(tmem_S0, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + off, 16, 1024),
+            mma_bf16(tmem, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + off, 16, 1024),
                      idesc_s, kk > 0);
           }
           mma_commit(bar_sfull);
+          mma_commit(bar_kempty);
         }
       }
       for (int j = 0; ok && j < plan.n_tiles; ++j) {
         if (j + 1 < plan.n_tiles) {
           const int jn = j + 1;
-          const int st = jn % kStages;
-          if (!mbar_wait(bar_kfull + 8 * st, (jn / kStages) & 1, a.status)) break;
+          const int st = jn % kKStages;
+          if (!mbar_wait(bar_kfull + 8 * st, (jn / kKStages) & 1, a.status)) break;
           tc_fence_after();
           const uint32_t kb = sK + st * L::tile;
-          const uint32_t sbuf = tmem_S0 + (jn & 1) * 128;
+          const uint32_t sbuf = tmem + (jn % kSBufs) * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
             mma_bf16(sbuf, sw128_desc(sQ + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
                      idesc_s, kk > 0);
           }
-          mma_commit(bar_sfull + 8 * (jn & 1));
+          mma_commit(bar_sfull + 8 * (jn % kSBufs));
+          mma_commit(bar_kempty + 8 * st);
         }
-        const int st = j % kStages;
+        const int st = j % kVStages;
         if (!mbar_wait(bar_pfull, j & 1, a.status)) break;
-        if (!mbar_wait(bar_vfull + 8 * st, (j / kStages) & 1, a.status)) break;
+        if (!mbar_wait(bar_vfull + 8 * st, (j / kVStages) & 1, a.status)) break;
         tc_fence_after();
         const uint32_t vb = sV + st * L::tile;
+        const uint32_t pcol = tmem + (j % kSBufs) * 128;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * kSubBytes + (kk & 3) * 32;
-          mma_bf16(tmem_O, sw128_desc(sP + aoff, 16, 1024),
-                   sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o, (j > 0 || kk > 0));
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16_tmem_a(tmem + kTmemO, pcol + kk * 8,
+                          sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o,
+                          (j > 0 || kk > 0));
         mma_commit(bar_odone);
-        mma_commit(bar_empty + 8 * st);
+        mma_commit(bar_vempty + 8 * st);
+        if (j + 1 == plan.n_tiles) mma_commit(bar_ofinal);
       }
       // every MMA this thread issued has finished before tensor memory is freed
       mma_commit(bar_idle);
@@ -408,114 +449,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
-    const int r = tid;                            // query row within the tile
+    const int hh = warp >> 2;                     // column half of the tile
+    const int r = (warp & 3) * 32 + lane;         // query row within the tile
     const bool real_row = r < rows;
     const int t = plan.t_min + (real_row ? r : rows - 1);
     const int wl = window_lo(t, a.block, a.window);
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float c = a.scale_log2;
-    float m_used = -INFINITY;  // scaled (log2) units
-    float l_sum = 0.f;
+    float m_used = -INFINITY;  // scaled (log2) units, identical in both halves
+    float l_half = 0.f;
     bool ok = true;
     for (int j = 0; j < plan.n_tiles; ++j) {
-      if (!mbar_wait(bar_sfull + 8 * (j & 1), (j >> 1) & 1, a.status)) { ok = false; break; }
+      const int sb = j % kSBufs;
+      if (!mbar_wait(bar_sfull + 8 * sb, (j / kSBufs) & 1, a.status)) { ok = false; break; }
       tc_fence_after();
       const int k0 = tile_key0(plan, j);
       const bool masked = tile_needs_mask(plan, k0, a.sink);
-      const uint32_t srow = tmem_S0 + (j & 1) * 128 + lane_base;
-      uint32_t s[BN];
-#pragma unroll
-      for (int q = 0; q < BN / 32; ++q) {
-        uint32_t* sq = s + q * 32;
-        FLUX_TMEM_LD32(srow + q * 32, sq);
+      const uint32_t scol = tmem + sb * 128 + hh * 64 + lane_base;
+      uint32_t s[64];
+      FLUX_TMEM_LD32(scol, s);
+      {
+        uint32_t* s2 = s + 32;
+        FLUX_TMEM_LD32(scol + 32, s2);
       }
       tmem_wait_ld();
       if (masked) {
+        const int kb = k0 + hh * 64;
 #pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          const int jk = k0 + i;
+        for (int i = 0; i < 64; ++i) {
+          const int jk = kb + i;
           const bool vis = (jk <= t) && (plan.fa || jk < a.sink || jk >= wl);
           if (!vis) s[i] = __float_as_uint(-INFINITY);
         }
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+      for (int i = 0; i < 64; i += 2)
+        mx = fmax3(mx, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+      // exchange half-row maxima with the other warpgroup
+      red[((j & 1) * 2 + hh) * 128 + r] = mx;
+      named_barrier_sync(1, kSoftmaxThreads);
+      mx = fmaxf(mx, red[((j & 1) * 2 + (hh ^ 1)) * 128 + r]);
       const float m_tile = mx * c;
-      const bool raise = (m_used == -INFINITY) ? (m_tile > -INFINITY)
-                                               : (m_tile > m_used + kRescaleThreshold);
-      // P_{j-1} V_{j-1} must be complete before O is rescaled or P is overwritten
-      if (j > 0) {
-        if (!mbar_wait(bar_odone, (j - 1) & 1, a.status)) { ok = false; break; }
-        tc_fence_after();
-      }
+      const bool bump = (m_used == -INFINITY) ? (m_tile > -INFINITY)
+                                              : (m_tile > m_used + kRescaleThreshold);
       float alpha = 1.f;
-      if (raise) {
+      if (bump) {
         alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_tile);
         m_used = m_tile;
-        l_sum *= alpha;
+        l_half *= alpha;
       }
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        const uint32_t orow = tmem_O + lane_base;
+      const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+      // P = exp2(S * c - m) as packed bf16 pairs; row sum of this half
+      uint32_t pk[32];
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
+      for (int w = 0; w < 32; ++w) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(s[2 * w]), c, -m_use));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(s[2 * w + 1]), c, -m_use));
+        l_half += p0 + p1;
+        pk[w] = pack_bf16x2(p0, p1);
+      }
+      // O rescale needs P_{j-1} V_{j-1} complete; tile j's s_full already implies that
+      // every MMA before S_j (P_{j-2} V_{j-2} and older) is complete, so o_done is at
+      // most one phase behind here.
+      if (j > 0 && __any_sync(0xffffffffu, bump)) {
+        if (!mbar_wait(bar_odone, (j - 1) & 1, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ocol = tmem + kTmemO + hh * DH + lane_base;
+#pragma unroll
+        for (int q = 0; q < DH / 32; ++q) {
           uint32_t ov[32];
-          FLUX_TMEM_LD32(orow + q * 32, ov);
+          FLUX_TMEM_LD32(ocol + q * 32, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          FLUX_TMEM_ST32(orow + q * 32, ov);
-        }
-        tmem_wait_st();
-      }
-      const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
-      // P = exp2(S * c - m), row sum, bf16 into the swizzled K-major P tile
-#pragma unroll
-      for (int sb = 0; sb < 2; ++sb) {
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = sb * 64 + cc * 8 + 2 * e;
-            const float p0 = fast_exp2(fmaf(__uint_as_float(s[i]), c, -m_use));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(s[i + 1]), c, -m_use));
-            l_sum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          const uint32_t addr = sP + sb * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128 +
-                                ((cc ^ (r & 7)) << 4);
-          sts128(addr, pk[0], pk[1], pk[2], pk[3]);
+          FLUX_TMEM_ST32(ocol + q * 32, ov);
         }
       }
+      // P over the first 64 columns of this S buffer: keys 64hh + 2w, 64hh + 2w + 1 in
+      // column 32hh + w
+      FLUX_TMEM_ST32(tmem + sb * 128 + hh * 32 + lane_base, pk);
+      tmem_wait_st();
       // keys past the valid length: zero their V rows (the cache there is unwritten)
-      if (k0 + BN > seq) {
-        const int st = j % kStages;
-        if (!mbar_wait(bar_vfull + 8 * st, (j / kStages) & 1, a.status)) { ok = false; break; }
+      if (k0 + BN > seq && hh < NCH) {
+        const int st = j % kVStages;
+        if (!mbar_wait(bar_vfull + 8 * st, (j / kVStages) & 1, a.status)) { ok = false; break; }
         if (k0 + r >= seq) {
+          const uint32_t vrow = sV + st * L::tile + hh * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-          for (int cch = 0; cch < NCH; ++cch) {
-            const uint32_t vrow = sV + st * L::tile + cch * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-            for (int x = 0; x < 8; ++x) sts128(vrow + x * 16, 0u, 0u, 0u, 0u);
-          }
+          for (int x = 0; x < 8; ++x) sts128(vrow + x * 16, 0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull);
     }
-    // epilogue: O / l -> bf16 -> global
-    if (ok && plan.n_tiles > 0 && mbar_wait(bar_odone, (plan.n_tiles - 1) & 1, a.status)) {
+    // epilogue: O / l -> bf16 -> global, each warpgroup its half of the columns
+    lsum[hh * 128 + r] = l_half;
+    named_barrier_sync(1, kSoftmaxThreads);
+    const float l_row = l_half + lsum[(hh ^ 1) * 128 + r];
+    if (ok && plan.n_tiles > 0 && mbar_wait(bar_ofinal, 0, a.status)) {
       tc_fence_after();
-      const float inv_l = 1.f / l_sum;
-      const uint32_t orow = tmem_O + lane_base;
-      uint16_t* dst = a.o + ((size_t(b) * a.n_q + row0 + r) * a.hq + h) * D;
+      const float inv_l = 1.f / l_row;
+      const uint32_t ocol = tmem + kTmemO + hh * DH + lane_base;
+      uint16_t* dst = a.o + ((size_t(b) * a.n_q + row0 + r) * a.hq + h) * D + hh * DH;
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = 0; q < DH / 32; ++q) {
         uint32_t ov[32];
-        FLUX_TMEM_LD32(orow + q * 32, ov);
+        FLUX_TMEM_LD32(ocol + q * 32, ov);
         tmem_wait_ld();
         if (real_row) {
 #pragma unroll
