@@ -5,33 +5,34 @@
 // read on the device from the layer's bit of the router's mask (Figure 2).
 //
 // One CTA computes one 128-query tile of one query head.  Roles (352 threads):
-//   warps 0-7  softmax, two warpgroups: warpgroup h (h = 0, 1) owns columns
-//              [64h, 64h + 64) of each 128-key tile for all 128 query rows (thread =
-//              one row in one half).  It reads its half of S = Q K^T from tensor
-//              memory (tcgen05.ld), masks boundary tiles, swaps half-row maxima with
-//              the other warpgroup through shared memory, runs the online softmax in
-//              registers (log2 domain; a stale row maximum raised only when the new
-//              maximum exceeds it by more than 2^8, and then O is rescaled in tensor
-//              memory), and writes P as bf16 back into tensor memory over its own S
-//              columns, where the P.V MMA reads it as its A operand.  At the end it
-//              normalises its half of the O row and stores it.
+//   warps 0-7  softmax, two warpgroups that ping-pong over the KV tiles: warpgroup g
+//              (g = 0, 1) takes the tiles j = g, g + 2, g + 4, ...  Thread = one
+//              query row.  For its tile it reads the row of S = Q K^T from tensor
+//              memory (tcgen05.ld), masks boundary tiles, runs the online softmax in
+//              registers (log2 domain; its own stale row maximum, raised only when
+//              the new maximum exceeds it by more than 2^8, and then its O is
+//              rescaled in tensor memory) and writes P as bf16 back into tensor
+//              memory over its S columns, where the P.V MMA reads it as the A
+//              operand.  The exponentials are taken against the current maximum in
+//              the same pass that finds the tile maximum; only a warp with a row
+//              whose maximum jumped re-reads the tile.  Each warpgroup accumulates its own O; at the end the two
+//              partial (max, sum, O) are merged per row, normalised and stored.
 //   warps 8-9  TMA producers (cp.async.bulk.tensor, 128-byte swizzle, no cluster, no
 //              multicast): warp 8 the Q tile once and K tiles into a 3-stage ring that
 //              is released as soon as each tile's S MMAs complete; warp 9 V tiles into
 //              a 2-stage ring released by the P.V MMAs.
 //   warp 10    MMA issuer (one thread): S_j = Q K_j^T (A, B from shared memory) into
-//              one of three S buffers in tensor memory, then O += P_j V_j with P_j
-//              read from tensor memory and V_j an MN-major shared-memory operand;
-//              completion is signalled with tcgen05.commit on mbarriers.  The warp
-//              also allocates and frees the 512 tensor-memory columns
-//              (S0 | S1 | S2 | O).
-// S_{j+1} is issued before P_j V_j, so the tensor cores compute the next scores while
-// the softmax warps work on the current ones; with three S buffers, the buffer S_{j+1}
-// lands in last held P_{j-2}, whose P.V MMA was issued two MMA groups earlier.
+//              the S buffer of warpgroup j % 2, O_{j%2} += P_j V_j with P_j read from
+//              tensor memory and V_j an MN-major shared-memory operand; completion is
+//              signalled with tcgen05.commit on mbarriers.  S_{j+2} is issued right
+//              after P_j V_j: this thread's MMAs execute in issue order, so P_j has
+//              been read before S_{j+2} overwrites it.  The warp also allocates and
+//              frees the 512 tensor-memory columns (S0 | S1 | O0 | O1).
+// While one warpgroup runs its exponentials the tensor cores serve the other one.
 //
 // Every mbarrier wait is bounded: on time-out the thread records FLUX_DEVICE_TIMEOUT
-// and leaves its loop; all roles meet at the final barrier, the producer first waits
-// for its copies in flight, the MMA thread for its MMAs, and the tensor memory is
+// and leaves its loop; all roles meet at the final barrier, the producers first wait
+// for their copies in flight, the MMA thread for its MMAs, and the tensor memory is
 // always freed.
 #include <cuda.h>
 #include <math.h>
@@ -51,11 +52,15 @@ constexpr int kKProducerWarp = 8;
 constexpr int kVProducerWarp = 9;
 constexpr int kMmaWarp = 10;
 constexpr int kThreads = 352;
-constexpr int kSBufs = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 384;           // O accumulator columns [384, 384 + D)
+constexpr uint32_t kTmemO = 256;           // O_g accumulator columns [256 + 128 g, + D)
 constexpr uint32_t kSubBytes = 128 * 128;  // one 64-column swizzled sub-tile of 128 rows
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 8 exponential pairs of a softmax row, this many go to the MUFU unit and the
+// rest to the polynomial on the FMA pipe.  Measured on B200 (Llama shape, 32K prompt):
+// 8/8 -> 8.09 ms, 6/8 -> 8.45 ms, 5/8 -> 8.70 ms: the softmax warps are bound by issue
+// and latency, not by MUFU throughput, so every exponential stays on MUFU.
+constexpr int kMufuPairsPer8 = 8;
 
 template <int D>
 struct Smem {
@@ -64,12 +69,12 @@ struct Smem {
   static constexpr uint32_t off_q = 0;
   static constexpr uint32_t off_k = off_q + tile;
   static constexpr uint32_t off_v = off_k + kKStages * tile;
-  static constexpr uint32_t off_red = off_v + kVStages * tile;  // float [2][2][128] maxima
-  static constexpr uint32_t off_lsum = off_red + 2 * 2 * 128 * 4;  // float [2][128]
-  static constexpr uint32_t off_bar = off_lsum + 2 * 128 * 4;
-  // q_full | k_full[3] | k_empty[3] | v_full[2] | v_empty[2] | s_full[3] | p_full |
-  // o_done | o_final | mma_idle
-  static constexpr int n_bars = 1 + 2 * kKStages + 2 * kVStages + kSBufs + 4;
+  static constexpr uint32_t off_ms = off_v + kVStages * tile;  // float [2][128] row maxima
+  static constexpr uint32_t off_ls = off_ms + 2 * 128 * 4;      // float [2][128] row sums
+  static constexpr uint32_t off_bar = off_ls + 2 * 128 * 4;
+  // q_full | k_full[3] | k_empty[3] | v_full[2] | v_empty[2] | s_full[2] | p_full[2] |
+  // o_done[2] | o_final | mma_idle
+  static constexpr int n_bars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2;
   static constexpr uint32_t off_tmem = off_bar + n_bars * 8;
   static constexpr uint32_t used = off_tmem + 16;
   // 1 KB slack to align the base; at least 116 KB so that a second CTA (which would
@@ -162,11 +167,6 @@ __device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
       : "memory");
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
@@ -295,19 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = base + L::off_q;
   const uint32_t sK = base + L::off_k;
   const uint32_t sV = base + L::off_v;
-  float* red = reinterpret_cast<float*>(smem + L::off_red);
-  float* lsum = reinterpret_cast<float*>(smem + L::off_lsum);
+  float* ms = reinterpret_cast<float*>(smem + L::off_ms);
+  float* ls = reinterpret_cast<float*>(smem + L::off_ls);
   const uint32_t bar0 = base + L::off_bar;
   const uint32_t bar_q = bar0;
   const uint32_t bar_kfull = bar0 + 8;                        // + 8 * K stage
   const uint32_t bar_kempty = bar_kfull + 8 * kKStages;
   const uint32_t bar_vfull = bar_kempty + 8 * kKStages;       // + 8 * V stage
   const uint32_t bar_vempty = bar_vfull + 8 * kVStages;
-  const uint32_t bar_sfull = bar_vempty + 8 * kVStages;       // + 8 * S buffer
-  const uint32_t bar_pfull = bar_sfull + 8 * kSBufs;
-  const uint32_t bar_odone = bar_pfull + 8;
-  const uint32_t bar_ofinal = bar_pfull + 16;
-  const uint32_t bar_idle = bar_pfull + 24;
+  const uint32_t bar_sfull = bar_vempty + 8 * kVStages;       // + 8 * warpgroup
+  const uint32_t bar_pfull = bar_sfull + 16;                  // + 8 * warpgroup
+  const uint32_t bar_odone = bar_pfull + 16;                  // + 8 * warpgroup
+  const uint32_t bar_ofinal = bar_odone + 16;
+  const uint32_t bar_idle = bar_ofinal + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_tmem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -337,9 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_vfull + 8 * s, 1);
       mbar_init(bar_vempty + 8 * s, 1);
     }
-    for (int s = 0; s < kSBufs; ++s) mbar_init(bar_sfull + 8 * s, 1);
-    mbar_init(bar_pfull, kSoftmaxThreads / 32);
-    mbar_init(bar_odone, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar_sfull + 8 * g, 1);
+      mbar_init(bar_pfull + 8 * g, 4);
+      mbar_init(bar_odone + 8 * g, 1);
+    }
     mbar_init(bar_ofinal, 1);
     mbar_init(bar_idle, 1);
     fence_barrier_init();
@@ -397,176 +399,237 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = make_idesc(BM, BN, false, false);
       constexpr uint32_t idesc_o = make_idesc(BM, D, false, true);
       bool ok = mbar_wait(bar_q, 0, a.status);
-      if (ok && plan.n_tiles > 0) {
-        ok = mbar_wait(bar_kfull, 0, a.status);
-        if (ok) {
-          tc_fence_after();
+      // S_j = Q K_j^T into the S buffer of warpgroup j % 2
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % kKStages;
+        if (!mbar_wait(bar_kfull + 8 * st, (j / kKStages) & 1, a.status)) return false;
+        tc_fence_after();
+        const uint32_t kb = sK + st * L::tile;
+        const uint32_t sbuf = tmem + (j & 1) * 128;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
-            mma_bf16(tmem, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + off, 16, 1024),
-                     idesc_s, kk > 0);
-          }
-          mma_commit(bar_sfull);
-          mma_commit(bar_kempty);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+          mma_bf16(sbuf, sw128_desc(sQ + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_s,
+                   kk > 0);
         }
-      }
+        mma_commit(bar_sfull + 8 * (j & 1));
+        mma_commit(bar_kempty + 8 * st);
+        return true;
+      };
+      if (ok && plan.n_tiles > 0) ok = issue_s(0);
+      if (ok && plan.n_tiles > 1) ok = issue_s(1);
       for (int j = 0; ok && j < plan.n_tiles; ++j) {
-        if (j + 1 < plan.n_tiles) {
-          const int jn = j + 1;
-          const int st = jn % kKStages;
-          if (!mbar_wait(bar_kfull + 8 * st, (jn / kKStages) & 1, a.status)) break;
-          tc_fence_after();
-          const uint32_t kb = sK + st * L::tile;
-          const uint32_t sbuf = tmem + (jn % kSBufs) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
-            mma_bf16(sbuf, sw128_desc(sQ + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
-                     idesc_s, kk > 0);
-          }
-          mma_commit(bar_sfull + 8 * (jn % kSBufs));
-          mma_commit(bar_kempty + 8 * st);
-        }
+        const int g = j & 1;
         const int st = j % kVStages;
-        if (!mbar_wait(bar_pfull, j & 1, a.status)) break;
         if (!mbar_wait(bar_vfull + 8 * st, (j / kVStages) & 1, a.status)) break;
+        if (!mbar_wait(bar_pfull + 8 * g, (j >> 1) & 1, a.status)) break;
         tc_fence_after();
         const uint32_t vb = sV + st * L::tile;
-        const uint32_t pcol = tmem + (j % kSBufs) * 128;
+        const uint32_t pcol = tmem + g * 128;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_tmem_a(tmem + kTmemO, pcol + kk * 8,
+          mma_bf16_tmem_a(tmem + kTmemO + g * 128, pcol + kk * 8,
                           sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o,
-                          (j > 0 || kk > 0));
-        mma_commit(bar_odone);
+                          (j >= 2 || kk > 0));
         mma_commit(bar_vempty + 8 * st);
-        if (j + 1 == plan.n_tiles) mma_commit(bar_ofinal);
+        // S_{j+2} overwrites P_j.  MMAs issued by this thread execute in issue order,
+        // so P_j V_j has read its operand before S_{j+2} writes the buffer.
+        if (j + 2 < plan.n_tiles && !issue_s(j + 2)) break;
       }
       // every MMA this thread issued has finished before tensor memory is freed
+      mma_commit(bar_ofinal);
       mma_commit(bar_idle);
       mbar_wait(bar_idle, 0, a.status);
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
-    const int hh = warp >> 2;                     // column half of the tile
+    const int g = warp >> 2;                      // warpgroup: tiles j = g (mod 2)
     const int r = (warp & 3) * 32 + lane;         // query row within the tile
     const bool real_row = r < rows;
     const int t = plan.t_min + (real_row ? r : rows - 1);
     const int wl = window_lo(t, a.block, a.window);
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t srow = tmem + g * 128 + lane_base;
+    const uint32_t orow = tmem + kTmemO + g * 128 + lane_base;
     const float c = a.scale_log2;
-    float m_used = -INFINITY;  // scaled (log2) units, identical in both halves
-    float l_half = 0.f;
+    float m_used = -INFINITY;  // scaled (log2) units
+    float l_sum = 0.f;
     bool ok = true;
-    for (int j = 0; j < plan.n_tiles; ++j) {
-      const int sb = j % kSBufs;
-      if (!mbar_wait(bar_sfull + 8 * sb, (j / kSBufs) & 1, a.status)) { ok = false; break; }
+    for (int j = g; j < plan.n_tiles; j += 2) {
+      if (!mbar_wait(bar_sfull + 8 * g, (j >> 1) & 1, a.status)) { ok = false; break; }
       tc_fence_after();
       const int k0 = tile_key0(plan, j);
       const bool masked = tile_needs_mask(plan, k0, a.sink);
-      const uint32_t scol = tmem + sb * 128 + hh * 64 + lane_base;
-      uint32_t s[64];
-      FLUX_TMEM_LD32(scol, s);
+      // Load 64 columns of the S row into s[] and apply the tile's mask.
+      auto load_half = [&](uint32_t (&s)[64], int half) {
+        FLUX_TMEM_LD32(srow + half * 64, s);
+        {
+          uint32_t* s2 = s + 32;
+          FLUX_TMEM_LD32(srow + half * 64 + 32, s2);
+        }
+        tmem_wait_ld();
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int jk = k0 + half * 64 + i;
+            const bool vis = (jk <= t) && (plan.fa || jk < a.sink || jk >= wl);
+            if (!vis) s[i] = __float_as_uint(-INFINITY);
+          }
+        }
+      };
+      auto max_half = [&](const uint32_t (&s)[64]) -> float {
+        float mx[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx[x] = __uint_as_float(s[x]);
+#pragma unroll
+        for (int i = 8; i < 64; i += 16)
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            mx[x] = fmax3(mx[x], __uint_as_float(s[i + x]), __uint_as_float(s[i + 8 + x]));
+        return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+      };
+      // P = exp2(S * c - m) of one half as packed bf16 pairs over columns
+      // [32 half, 32 half + 32) of the buffer (keys 2w, 2w + 1 in column w); returns the
+      // half's row sum.  The S values there were consumed before this store.
+      auto exp_half = [&](const uint32_t (&s)[64], int half, float m_use) -> float {
+        const uint64_t c2 = f2_pack(c, c);
+        const uint64_t nm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[32];
+#pragma unroll
+        for (int w = 0; w < 32; ++w) {
+          const uint64_t x2 =
+              f2_fma(f2_pack(__uint_as_float(s[2 * w]), __uint_as_float(s[2 * w + 1])), c2, nm2);
+          uint64_t p2;
+          if ((w & 7) >= kMufuPairsPer8) {
+            p2 = exp2_poly_f2(x2);  // on the FMA pipe
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_mufu(x0), ex2_mufu(x1));
+          }
+          acc[w & 3] = f2_add(acc[w & 3], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          pk[w] = pack_bf16x2(p0, p1);
+        }
+        FLUX_TMEM_ST32(srow + half * 32, pk);
+        const uint64_t sum2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float s0, s1;
+        f2_unpack(sum2, s0, s1);
+        return s0 + s1;
+      };
+      // Fast path: exponentials against the current stale maximum, one TMEM read of S.
+      // Any row of the warp whose maximum moved by more than the threshold (and the
+      // first tile) sends the warp to the slow path, which recomputes the tile.
+      float mrow, lpart = 0.f;
+      bool slow;
       {
-        uint32_t* s2 = s + 32;
-        FLUX_TMEM_LD32(scol + 32, s2);
-      }
-      tmem_wait_ld();
-      if (masked) {
-        const int kb = k0 + hh * 64;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const int jk = kb + i;
-          const bool vis = (jk <= t) && (plan.fa || jk < a.sink || jk >= wl);
-          if (!vis) s[i] = __float_as_uint(-INFINITY);
+        uint32_t s[64];
+        load_half(s, 0);
+        mrow = max_half(s);
+        slow = __any_sync(0xffffffffu, m_used == -INFINITY || mrow * c > m_used + kRescaleThreshold);
+        if (!slow) {
+          lpart = exp_half(s, 0, m_used);
+          load_half(s, 1);
+          const float m1 = max_half(s);
+          mrow = fmaxf(mrow, m1);
+          slow = __any_sync(0xffffffffu, m1 * c > m_used + kRescaleThreshold);
+          if (!slow) lpart += exp_half(s, 1, m_used);
+        } else {
+          load_half(s, 1);
+          mrow = fmaxf(mrow, max_half(s));
         }
       }
-      float mx = -INFINITY;
+      if (slow) {
+        const float m_tile = mrow * c;
+        const bool bump = (m_used == -INFINITY) ? (m_tile > -INFINITY)
+                                                : (m_tile > m_used + kRescaleThreshold);
+        float alpha = 1.f;
+        if (bump) {
+          alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_tile);
+          m_used = m_tile;
+          l_sum *= alpha;
+        }
+        // O_g was last written by P_{j-2} V_{j-2}; the commit that signalled S_j
+        // covers it, so it has completed
+        if (j >= 2 && __any_sync(0xffffffffu, bump)) {
 #pragma unroll
-      for (int i = 0; i < 64; i += 2)
-        mx = fmax3(mx, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-      // exchange half-row maxima with the other warpgroup
-      red[((j & 1) * 2 + hh) * 128 + r] = mx;
-      named_barrier_sync(1, kSoftmaxThreads);
-      mx = fmaxf(mx, red[((j & 1) * 2 + (hh ^ 1)) * 128 + r]);
-      const float m_tile = mx * c;
-      const bool bump = (m_used == -INFINITY) ? (m_tile > -INFINITY)
-                                              : (m_tile > m_used + kRescaleThreshold);
-      float alpha = 1.f;
-      if (bump) {
-        alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_tile);
-        m_used = m_tile;
-        l_half *= alpha;
-      }
-      const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
-      // P = exp2(S * c - m) as packed bf16 pairs; row sum of this half
-      uint32_t pk[32];
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t ov[32];
+            FLUX_TMEM_LD32(orow + q * 32, ov);
+            tmem_wait_ld();
 #pragma unroll
-      for (int w = 0; w < 32; ++w) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(s[2 * w]), c, -m_use));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(s[2 * w + 1]), c, -m_use));
-        l_half += p0 + p1;
-        pk[w] = pack_bf16x2(p0, p1);
-      }
-      // O rescale needs P_{j-1} V_{j-1} complete; tile j's s_full already implies that
-      // every MMA before S_j (P_{j-2} V_{j-2} and older) is complete, so o_done is at
-      // most one phase behind here.
-      if (j > 0 && __any_sync(0xffffffffu, bump)) {
-        if (!mbar_wait(bar_odone, (j - 1) & 1, a.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t ocol = tmem + kTmemO + hh * DH + lane_base;
-#pragma unroll
-        for (int q = 0; q < DH / 32; ++q) {
-          uint32_t ov[32];
-          FLUX_TMEM_LD32(ocol + q * 32, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          FLUX_TMEM_ST32(ocol + q * 32, ov);
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            FLUX_TMEM_ST32(orow + q * 32, ov);
+          }
+        }
+        const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+        lpart = 0.f;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t s[64];
+          load_half(s, half);
+          lpart += exp_half(s, half, m_use);
         }
       }
-      // P over the first 64 columns of this S buffer: keys 64hh + 2w, 64hh + 2w + 1 in
-      // column 32hh + w
-      FLUX_TMEM_ST32(tmem + sb * 128 + hh * 32 + lane_base, pk);
+      l_sum += lpart;
       tmem_wait_st();
       // keys past the valid length: zero their V rows (the cache there is unwritten)
-      if (k0 + BN > seq && hh < NCH) {
+      if (k0 + BN > seq) {
         const int st = j % kVStages;
         if (!mbar_wait(bar_vfull + 8 * st, (j / kVStages) & 1, a.status)) { ok = false; break; }
         if (k0 + r >= seq) {
-          const uint32_t vrow = sV + st * L::tile + hh * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-          for (int x = 0; x < 8; ++x) sts128(vrow + x * 16, 0u, 0u, 0u, 0u);
+          for (int cch = 0; cch < NCH; ++cch) {
+            const uint32_t vrow = sV + st * L::tile + cch * kSubBytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) sts128(vrow + x * 16, 0u, 0u, 0u, 0u);
+          }
         }
         fence_proxy_async_smem();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull);
+      if (lane == 0) mbar_arrive(bar_pfull + 8 * g);
     }
-    // epilogue: O / l -> bf16 -> global, each warpgroup its half of the columns
-    lsum[hh * 128 + r] = l_half;
+    // epilogue: merge the two warpgroups' (max, sum, O), normalise, store; warpgroup g
+    // writes output columns [g D/2, (g + 1) D/2)
+    ms[g * 128 + r] = m_used;
+    ls[g * 128 + r] = l_sum;
     named_barrier_sync(1, kSoftmaxThreads);
-    const float l_row = l_half + lsum[(hh ^ 1) * 128 + r];
+    const bool two = plan.n_tiles > 1;
+    const float m0 = ms[r], m1 = two ? ms[128 + r] : -INFINITY;
+    const float M = fmaxf(m0, m1);
+    const float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M);
+    const float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M);
+    const float inv_l = 1.f / (a0 * ls[r] + (two ? a1 * ls[128 + r] : 0.f));
     if (ok && plan.n_tiles > 0 && mbar_wait(bar_ofinal, 0, a.status)) {
       tc_fence_after();
-      const float inv_l = 1.f / l_row;
-      const uint32_t ocol = tmem + kTmemO + hh * DH + lane_base;
-      uint16_t* dst = a.o + ((size_t(b) * a.n_q + row0 + r) * a.hq + h) * D + hh * DH;
+      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+      const uint32_t o0 = tmem + kTmemO + lane_base + g * DH;
+      uint16_t* dst = a.o + ((size_t(b) * a.n_q + row0 + r) * a.hq + h) * D + g * DH;
 #pragma unroll
       for (int q = 0; q < DH / 32; ++q) {
-        uint32_t ov[32];
-        FLUX_TMEM_LD32(ocol + q * 32, ov);
+        uint32_t x0[32], x1[32];
+        FLUX_TMEM_LD32(o0 + q * 32, x0);
+        if (two) {
+          FLUX_TMEM_LD32(o0 + 128 + q * 32, x1);
+        }
         tmem_wait_ld();
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          f[i] = two ? fmaf(__uint_as_float(x0[i]), w0, __uint_as_float(x1[i]) * w1)
+                     : __uint_as_float(x0[i]) * w0;
         if (real_row) {
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ov[8 * x + 0]) * inv_l, __uint_as_float(ov[8 * x + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(ov[8 * x + 2]) * inv_l, __uint_as_float(ov[8 * x + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(ov[8 * x + 4]) * inv_l, __uint_as_float(ov[8 * x + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(ov[8 * x + 6]) * inv_l, __uint_as_float(ov[8 * x + 7]) * inv_l);
+            w.x = pack_bf16x2(f[8 * x + 0], f[8 * x + 1]);
+            w.y = pack_bf16x2(f[8 * x + 2], f[8 * x + 3]);
+            w.z = pack_bf16x2(f[8 * x + 4], f[8 * x + 5]);
+            w.w = pack_bf16x2(f[8 * x + 6], f[8 * x + 7]);
             *reinterpret_cast<uint4*>(dst + q * 32 + x * 8) = w;
           }
         }
