@@ -4,7 +4,9 @@ prefill + FA/SA decode) on B200.
 Main line (`value`): decode tokens/s of the Llama-3.1-8B attention shape serving 16
 sequences at a 32768-token context, 32 layers of which a fixed seeded 16 run SA
 (sink 128 + window 2048, block 128).  One step = one decode token for every sequence:
-per layer a KV append and an FA- or SA-routed split-KV decode.  The same run also
+per layer a KV append and an FA- or SA-routed split-KV decode, the 32 layers captured
+once as a CUDA graph and replayed per step (the eager, launch-by-launch number is
+reported beside it, and its FA decode launches give the HBM roofline).  The same run also
 times the prefill phase (router + 32 x (KV append + FA/SA prefill) of an 8192-token
 Llama-shaped prompt with router-chosen routes) and the decode step at every SA-layer
 fraction of the routing mix.  Protocol: W warm-up then K timed steps (default 10 and
@@ -141,18 +143,26 @@ def dist_setup(n_gpus: int):
     return world, rank, local
 
 
-def barrier(world):
+def barrier(world, device="cuda"):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if device == "cuda":
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """Largest value over the ranks (the slowest rank's time decides a replica run)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_tokens_per_s(world: int, tokens_per_rank: int, steps: int, t_ms: float) -> float:
+    """Whole-job throughput of N independent replicas: every rank processes its own
+    tokens_per_rank per step; the job takes as long as its slowest rank (t_ms)."""
+    return world * tokens_per_rank * steps / (t_ms / 1e3)
 
 
 def blas_threads() -> int:
@@ -432,13 +442,12 @@ def run_flux(args, world, rank, local):
         db.step(fa_events=fa_events)
     end.record()
     barrier(world)
-    clocks = sampler.stop()
     st = flux.flux_get_device_status()
     if st:
         raise RuntimeError(f"device status {st:#x} after the decode steps")
     t_ms = max_over_ranks(start.elapsed_time(end), world)
     ms_step = t_ms / args.steps
-    value = world * w.batch * args.steps / (t_ms / 1e3)
+    value = replica_tokens_per_s(world, w.batch, args.steps, t_ms)
     fa_ms = elapsed_ms(fa_events)
     # the timed steps run contexts 32769 .. 32768 + K; take the mean context
     T_mean = w.seq + (args.steps + 1) / 2.0
@@ -454,6 +463,32 @@ def run_flux(args, world, rank, local):
     sa_bytes = decode_bytes_per_layer(w, cfg, int(round(T_mean)), False)
     step_bytes = sum(decode_bytes_per_layer(w, cfg, int(round(T_mean)), fa) for fa in db.fa)
 
+    # ---------------- decode as one CUDA graph per step (the headline number)
+    from sparse_attention_layer_b200.runtime import DecodeStepGraph
+    db.reset()
+    graph = DecodeStepGraph(db.model, db.q, db.k_new, db.v_new, db.o)
+    db.reset()
+    for _ in range(args.warmup):  # warm-up replays outside the timed region
+        graph.replay()
+    db.reset()
+    barrier(world)
+    gs = torch.cuda.Event(enable_timing=True)
+    ge = torch.cuda.Event(enable_timing=True)
+    gs.record()
+    for _ in range(args.steps):
+        graph.replay()
+    ge.record()
+    barrier(world)
+    clocks = sampler.stop()  # sampled over the eager and the graph timed regions
+    tg_ms = max_over_ranks(gs.elapsed_time(ge), world)
+    eager = {"value": value, "ms_per_step": ms_step,
+             "what": "the same steps as 4 x 32 separate launches from Python"}
+    value = replica_tokens_per_s(world, w.batch, args.steps, tg_ms)
+    ms_step = tg_ms / args.steps
+    st = flux.flux_get_device_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} after the graph decode steps")
+
     # ---------------- decode: end to end from pinned host buffers
     q_h = db.q.cpu().pin_memory()
     k_h = db.k_new.cpu().pin_memory()
@@ -468,16 +503,16 @@ def run_flux(args, world, rank, local):
         db.q.copy_(q_h, non_blocking=True)
         db.k_new.copy_(k_h, non_blocking=True)
         db.v_new.copy_(v_h, non_blocking=True)
-        db.step()
+        graph.replay()
         o_h.copy_(db.o, non_blocking=True)
     e2.record()
     barrier(world)
     t2 = max_over_ranks(s2.elapsed_time(e2), world)
-    e2e = {"value": world * w.batch * args.steps / (t2 / 1e3), "unit": "tokens/s",
+    e2e = {"value": replica_tokens_per_s(world, w.batch, args.steps, t2), "unit": "tokens/s",
            "h2d_bytes_per_step": (q_h.numel() + k_h.numel() + v_h.numel()) * 2,
            "d2h_bytes_per_step": o_h.numel() * 2,
            "what": "per step: pinned-host q, k_new, v_new for all 32 layers copied in, the "
-                   "32-layer decode step, outputs of all layers copied out"}
+                   "captured 32-layer decode step replayed, outputs of all layers copied out"}
 
     # ---------------- routing mix: decode step time vs SA-layer fraction
     mix = {}
@@ -487,12 +522,12 @@ def run_flux(args, world, rank, local):
         n_sa = int(round(frac * w.n_layers))
         db.set_sa_layers(perm_sa[:n_sa])
         db.reset()
-        db.step()
+        graph.replay()
         barrier(world)
         a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(n_mix_steps):
-            db.step()
+            graph.replay()
         b.record()
         barrier(world)
         ms = max_over_ranks(a.elapsed_time(b), world) / n_mix_steps
@@ -502,7 +537,7 @@ def run_flux(args, world, rank, local):
     for v in mix.values():
         v["speedup_vs_all_fa"] = base / v["ms_per_step"]
     db.set_sa_layers(db.sa_layers)
-    del db
+    del graph, db
     torch.cuda.empty_cache()
 
     # ---------------- prefill phase (Llama shape, 8192 tokens, router-chosen routes)
@@ -564,7 +599,7 @@ def run_flux(args, world, rank, local):
         "decode_step": {"algorithmic_gb_per_step": step_bytes / 1e9,
                         "step_gb_per_s": step_bytes / (ms_step / 1e3) / 1e9,
                         "fa_layer_bytes": fa_bytes, "sa_layer_bytes": sa_bytes},
-        "cpu_baseline": cpu, "e2e": e2e,
+        "cpu_baseline": cpu, "e2e": e2e, "decode_eager": eager,
         "gpu_launches": w.n_layers * 4 * args.steps, "clocks": clocks,
         "prefill": prefill, "routing_mix": mix,
     }

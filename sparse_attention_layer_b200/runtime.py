@@ -56,3 +56,26 @@ class HybridAttention:
         flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, k_new, v_new)
         flux.flux_decode(self.cfg, layer, self.fa_mask, q, c.k, c.v, c.seq_len, out,
                          self.workspace)
+
+
+class DecodeStepGraph:
+    """One decode step over every layer (KV append + FA/SA decode per layer) captured in
+    a CUDA graph and replayed once per generated token.
+
+    Capture is possible because no call allocates, synchronises or reads device state
+    on the host: routes come from the device-side mask and lengths from seq_len, which
+    the captured appends advance on every replay.  q, k_new, v_new and o are the
+    static input/output buffers ([L][B][Hq][d], [L][B][1][Hkv][d] twice, [L][B][Hq][d]);
+    refill them in place between replays.  Run one eager step first (per-device
+    one-time set-up of the library happens outside the capture).
+    """
+
+    def __init__(self, model: HybridAttention, q, k_new, v_new, o):
+        self.buffers = (q, k_new, v_new, o)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            for layer in range(len(model.caches)):
+                model.decode_layer(layer, q[layer], k_new[layer], v_new[layer], o[layer])
+
+    def replay(self):
+        self.graph.replay()

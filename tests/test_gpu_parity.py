@@ -315,3 +315,41 @@ def test_decode_llama_full_size():
     ctx = [w.seq] * w.batch
     _decode_case(cfg, ctx, [True] * w.batch, 1, seed=1000, capacity=w.capacity(), layer=3)
     _decode_case(cfg, ctx, [False] * w.batch, 2, seed=1001, capacity=w.capacity(), layer=4)
+
+
+def test_decode_graph_replay_matches_eager():
+    """A decode step captured as a CUDA graph replays to the outputs of the eager calls
+    (lengths and routes are read on the device, so the graph serves every step)."""
+    from sparse_attention_layer_b200.runtime import DecodeStepGraph, HybridAttention
+    cfg = AttnCfg(3, 8, 2, 128, 128, 128, 256)
+    batch, ctx, steps = 3, 700, 4
+    mask = mask_words(batch, 3, [[0], [0, 2], []]).cuda()
+    models = [HybridAttention(cfg, batch, ctx + steps, "cuda") for _ in range(2)]
+    for m in models:
+        m.set_mask(mask)
+        for layer, c in enumerate(m.caches):
+            c.k.copy_(inputs.normal_bf16(c.k.shape, 50 + layer).cuda())
+            c.v.copy_(inputs.normal_bf16(c.v.shape, 60 + layer).cuda())
+            c.seq_len.fill_(ctx)
+    q = torch.zeros(3, batch, 8, 128, dtype=torch.bfloat16, device="cuda")
+    kn = torch.zeros(3, batch, 1, 2, 128, dtype=torch.bfloat16, device="cuda")
+    vn = torch.zeros_like(kn)
+    o = torch.zeros_like(q)
+    eager_m, graph_m = models
+    # one eager step on the graph model first (one-time set-up), then undo its append
+    for layer in range(3):
+        graph_m.decode_layer(layer, q[layer], kn[layer], vn[layer], o[layer])
+    for c in graph_m.caches:
+        c.seq_len.fill_(ctx)
+    g = DecodeStepGraph(graph_m, q, kn, vn, o)
+    for step in range(steps):
+        q.copy_(inputs.normal_bf16(q.shape, 70 + step).cuda())
+        kn.copy_(inputs.normal_bf16(kn.shape, 80 + step).cuda())
+        vn.copy_(inputs.normal_bf16(vn.shape, 90 + step).cuda())
+        o_e = torch.empty_like(o)
+        for layer in range(3):
+            eager_m.decode_layer(layer, q[layer], kn[layer], vn[layer], o_e[layer])
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_e), f"step {step}"
+    assert [int(c.seq_len[0]) for c in graph_m.caches] == [ctx + steps] * 3
