@@ -290,3 +290,56 @@ def kv_append(k_cache: np.ndarray, v_cache: np.ndarray, seq_len: np.ndarray,
             v_out[b, :, start + i, :] = v_new[b, i]
         len_out[b] = start + n_new
     return k_out, v_out, len_out, overflow
+
+
+# --------------------------------------------------------------------------------------
+# SA-layer KV eviction: sink rows plus a ring of recent rows (Tables 15/16 report the
+# persistent decode-time KV saving of layers routed to SA)
+# --------------------------------------------------------------------------------------
+
+
+def ring_slot(p, sink: int, ring_rows: int):
+    """Physical row of logical position p in an SA ring cache of sink + ring_rows rows:
+    sink positions stay in place, later positions cycle through the ring."""
+    p = np.asarray(p, dtype=np.int64)
+    return np.where(p < sink, p, sink + (p - sink) % ring_rows)
+
+
+def ring_retained_positions(seq_len: int, sink: int, ring_rows: int) -> np.ndarray:
+    """Logical positions an SA ring cache holds after seq_len rows were written: the sink
+    rows and the last ring_rows positions past the sink."""
+    head = np.arange(min(sink, seq_len), dtype=np.int64)
+    tail = np.arange(max(sink, seq_len - ring_rows), seq_len, dtype=np.int64)
+    return np.concatenate([head, tail])
+
+
+def kv_compact_ring(k_cache: np.ndarray, v_cache: np.ndarray, seq_len: np.ndarray,
+                    sink: int, ring_rows: int):
+    """Move a full cache [B][Hkv][cap][d] into ring caches [B][Hkv][sink + ring_rows][d]:
+    every retained position p goes to ring_slot(p).  Slots that hold no position stay
+    zero here (their content is unspecified in the library)."""
+    batch, hkv, _, d = k_cache.shape
+    k_ring = np.zeros((batch, hkv, sink + ring_rows, d), dtype=k_cache.dtype)
+    v_ring = np.zeros_like(k_ring)
+    for b in range(batch):
+        pos = ring_retained_positions(int(seq_len[b]), sink, ring_rows)
+        slots = ring_slot(pos, sink, ring_rows)
+        for h in range(hkv):
+            k_ring[b, h, slots] = k_cache[b, h, pos]
+            v_ring[b, h, slots] = v_cache[b, h, pos]
+    return k_ring, v_ring
+
+
+def kv_append_ring(k_ring: np.ndarray, v_ring: np.ndarray, seq_len: np.ndarray,
+                   k_new: np.ndarray, v_new: np.ndarray, sink: int, ring_rows: int):
+    """Append n rows per sequence at logical positions [seq_len, seq_len + n) into ring
+    caches and advance seq_len (rings never run out of room)."""
+    k_out, v_out = k_ring.copy(), v_ring.copy()
+    len_out = np.array(seq_len, dtype=np.int64).copy()
+    for b in range(len(len_out)):
+        for i in range(k_new.shape[1]):
+            slot = int(ring_slot(len_out[b] + i, sink, ring_rows))
+            k_out[b, :, slot] = k_new[b, i]
+            v_out[b, :, slot] = v_new[b, i]
+        len_out[b] += k_new.shape[1]
+    return k_out, v_out, len_out

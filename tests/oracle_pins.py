@@ -282,10 +282,45 @@ def check_router_error_bound(orc):
     assert (bound64 < bound32 * 2.0 ** -28).all()
 
 
+def check_ring_keeps_every_visible_key(orc):
+    """For every length T, the keys an SA decode query at T - 1 can see are all retained
+    by a ring of `window` rows, each in a slot of its own (no retained key is evicted
+    while still visible); a ring one row shorter loses one for some T."""
+    for block, sink, window in ((64, 64, 256), (128, 128, 2048), (64, 0, 128), (64, 128, 64)):
+        for T in range(1, sink + 3 * window + 2 * block, 5 if window > 512 else 1):
+            vis = np.nonzero(orc.sa_key_visible(T - 1, np.arange(T), block, sink, window))[0]
+            kept = set(orc.ring_retained_positions(T, sink, window).tolist())
+            assert set(vis.tolist()) <= kept, (block, sink, window, T)
+            slots = orc.ring_slot(vis, sink, window)
+            assert len(set(slots.tolist())) == len(vis)
+        lost = False
+        for T in range(1, sink + 3 * window + 2 * block):
+            vis = np.nonzero(orc.sa_key_visible(T - 1, np.arange(T), block, sink, window))[0]
+            if not set(vis.tolist()) <= set(orc.ring_retained_positions(T, sink, window - 1).tolist()):
+                lost = True
+                break
+        assert lost, (block, sink, window)
+
+
+def check_ring_placement_hand_example(orc):
+    """sink 2, ring 3, 9 positions written: slots 0, 1 hold positions 0, 1; the ring
+    holds positions 6, 7, 8 at slots 2 + (6-2)%3 = 3, 2 + 5%3 = 4, 2 + 6%3 = 2."""
+    assert orc.ring_slot([0, 1, 2, 3, 4, 5, 6, 7, 8], 2, 3).tolist() == [0, 1, 2, 3, 4, 2, 3, 4, 2]
+    assert orc.ring_retained_positions(9, 2, 3).tolist() == [0, 1, 6, 7, 8]
+    k = np.arange(9, dtype=float).reshape(1, 1, 9, 1) + 1
+    kr, vr = orc.kv_compact_ring(k, k, np.array([9]), 2, 3)
+    assert kr[0, 0, :, 0].tolist() == [1, 2, 9, 7, 8]
+    # appending position 9 overwrites slot 2 + 7 % 3 = 3 (position 6, no longer needed)
+    k2, v2, s2 = orc.kv_append_ring(kr, vr, np.array([9]), np.full((1, 1, 1, 1), 10.0),
+                                    np.full((1, 1, 1, 1), 10.0), 2, 3)
+    assert k2[0, 0, :, 0].tolist() == [1, 2, 9, 10, 8] and s2.tolist() == [10]
+
+
 ALL_CHECKS = [
     check_attention_vs_library, check_attention_closed_forms, check_softmax_rows,
     check_sa_counts_golden, check_sa_count_closed_form, check_sa_covers_fa,
     check_sa_token_reading_close, check_sa_key_blocks, check_decode_is_prefill_row,
     check_kv_append, check_router_golden, check_pool_indices, check_omega_pages,
-    check_router_error_bound,
+    check_router_error_bound, check_ring_keeps_every_visible_key,
+    check_ring_placement_hand_example,
 ]

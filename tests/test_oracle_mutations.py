@@ -34,6 +34,9 @@ MUTATIONS = {
     "append_off_by_one": ("k_out[b, :, start + i, :] = k_new[b, i]",
                           "k_out[b, :, start + i + 1, :] = k_new[b, i]"),
     "append_no_advance": ("len_out[b] = start + n_new", "len_out[b] = start"),
+    "ring_slot_offset": ("sink + (p - sink) % ring_rows)", "(p - sink) % ring_rows)"),
+    "ring_keeps_too_few": ("np.arange(max(sink, seq_len - ring_rows), seq_len",
+                           "np.arange(max(sink, seq_len - ring_rows + 1), seq_len"),
 }
 
 
