@@ -63,6 +63,7 @@ typedef enum flux_status {
 #define FLUX_DEVICE_CAPACITY 0x1u /* a kv_append would pass the capacity; skipped */
 #define FLUX_DEVICE_TIMEOUT 0x2u  /* a pipeline wait ran out of time; output invalid */
 #define FLUX_DEVICE_BAD_LENGTH 0x4u /* seq_len < n_q in prefill, or seq_len > capacity */
+#define FLUX_DEVICE_RING_ROUTE 0x8u /* flux_decode_ring saw a sequence routed to FA */
 
 /* Attention geometry of one model; the same struct serves every layer. */
 typedef struct flux_attn_cfg {
@@ -184,6 +185,42 @@ int flux_decode_static(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* 
                        const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
                        const int32_t* seq_len, int32_t batch, int32_t capacity, uint16_t* o,
                        void* stream);
+
+/*
+ * SA-layer KV eviction (the persistent decode-time KV saving of layers routed to SA,
+ * Tables 15/16).  An SA decode query only reads the sink rows and at most `window`
+ * recent rows, so after prefill an SA layer's cache can shrink to a ring cache of
+ * sink + ring_rows rows per (sequence, KV head), ring_rows >= window: position p < sink
+ * stays in row p, position p >= sink lives in row sink + (p - sink) % ring_rows.
+ * seq_len keeps counting logical positions.  Layout [batch][n_kv_heads][sink +
+ * ring_rows][head_dim] bf16.
+ *
+ * flux_kv_compact_ring -- copy the retained rows (positions [0, min(sink, seq_len))
+ *   and [max(sink, seq_len - ring_rows), seq_len)) of a full cache
+ *   [batch][n_kv_heads][capacity][head_dim] to their ring rows.  Other ring rows are
+ *   left as they were.  seq_len[b] > capacity sets FLUX_DEVICE_BAD_LENGTH.
+ */
+int flux_kv_compact_ring(const flux_attn_cfg* cfg, const uint16_t* k_cache,
+                         const uint16_t* v_cache, int32_t capacity, const int32_t* seq_len,
+                         int32_t batch, uint16_t* k_ring, uint16_t* v_ring, int32_t ring_rows,
+                         void* stream);
+
+/* flux_kv_append_ring -- flux_kv_append into a ring cache: rows for positions
+ * [seq_len[b], seq_len[b] + n_new) go to their ring rows (n_new <= ring_rows) and
+ * seq_len[b] += n_new; a ring never runs out of room. */
+int flux_kv_append_ring(const flux_attn_cfg* cfg, uint16_t* k_ring, uint16_t* v_ring,
+                        int32_t* seq_len, int32_t batch, int32_t ring_rows,
+                        const uint16_t* k_new, const uint16_t* v_new, int32_t n_new,
+                        void* stream);
+
+/* flux_decode_ring -- flux_decode of an SA layer over ring caches: same visible keys,
+ * same split plan and arithmetic as flux_decode over the full cache, so the results
+ * are identical.  A sequence routed to FA writes zeros and sets
+ * FLUX_DEVICE_RING_ROUTE (a ring holds only what SA reads). */
+int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                     const uint16_t* q, const uint16_t* k_ring, const uint16_t* v_ring,
+                     const int32_t* seq_len, int32_t batch, int32_t ring_rows, uint16_t* o,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * flux_sa_block_ranges -- the SA key-block set of each query block, as the kernels

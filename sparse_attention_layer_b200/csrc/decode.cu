@@ -56,27 +56,52 @@ struct DecodeArgs {
   int batch, capacity, hkv, block, sink, window;
   float scale_log2;  // log2(e) / sqrt(d)
   int min_splits;    // splits per (sequence, KV head) that give every SM 2 items
+  int ring_rows;     // 0: contiguous cache; > 0: SA ring cache of sink + ring_rows rows
+  int rows;          // physical rows per (sequence, KV head)
   float* ws_acc;     // [B][Hkv][kDecMaxSplits][G][D]
   float2* ws_ml;     // [B][Hkv][kDecMaxSplits][G] = (max, sum)
   uint16_t* o;
   unsigned* status;
 };
 
-// The visible keys of sequence b's decode query, flattened: virtual key v maps to
-// position v when v < len0, else to lo1 + (v - len0).
+// The visible keys of sequence b's decode query, flattened in position order and laid
+// out in up to three physically contiguous pieces: [0, len0) (sink, or everything in a
+// contiguous cache's merged case), then [start1, start1 + len1) and
+// [start2, start2 + len2) (the window; two pieces when it wraps around a ring cache).
 struct Plan {
-  int len0, lo1, n_vis, n_split, chunk;
+  int n_vis, n_split, chunk;
+  int len0, start1, len1, start2;
 };
 
 __device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
-  Plan p{0, 0, 0, 0, 1};
+  Plan p{0, 0, 1, 0, 0, 0, 0};
   const int T = a.seq_len[b];
   if (T <= 0 || T > a.capacity) return p;
   const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
+  if (a.ring_rows > 0 && fa) return p;  // a ring cache only holds what SA reads
   const KeyRanges r = visible_key_ranges(T - 1, fa, a.block, a.sink, a.window);
-  p.len0 = r.hi0 - r.lo0;
-  p.lo1 = r.lo1;
-  p.n_vis = p.len0 + (r.hi1 - r.lo1);
+  if (a.ring_rows == 0) {
+    p.len0 = r.hi0 - r.lo0;
+    p.start1 = r.lo1;
+    p.len1 = r.hi1 - r.lo1;
+  } else {
+    // positions below the sink stay in place; position q >= sink lives in slot
+    // sink + (q - sink) mod ring_rows
+    const int R = a.ring_rows;
+    if (r.lo1 == 0) {  // the window reaches key 0: keys [0, T), and T - sink <= window <= R
+      p.len0 = min(T, a.sink);
+      p.start1 = a.sink;
+      p.len1 = max(0, T - a.sink);
+    } else {
+      p.len0 = r.hi0;
+      const int L = r.hi1 - r.lo1;
+      const int s0 = (r.lo1 - a.sink) % R;
+      p.start1 = a.sink + s0;
+      p.len1 = min(L, R - s0);
+      p.start2 = a.sink;
+    }
+  }
+  p.n_vis = (r.hi0 - r.lo0) + (r.hi1 - r.lo1);
   // splits: enough items for every SM (min_splits), at most kDecMaxChunk keys each
   // when the split budget allows, never fewer than kDecMinChunk keys.
   const int by_min = (p.n_vis + kDecMinChunk - 1) / kDecMinChunk;
@@ -91,8 +116,8 @@ __device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
 
 struct Item {
   int b, kvh, split;
-  int a0, na;  // first piece: positions [a0, a0 + na)
-  int b0, nb;  // second piece: positions [b0, b0 + nb)
+  int v0, v1;  // this split's virtual keys
+  Plan p;
 };
 
 // Item idx of the flattened (sequence, KV head, split) list; prefix[b] counts the
@@ -105,42 +130,48 @@ __device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix, 
   }
   Item it;
   it.b = lo;
-  const Plan p = make_plan(a, lo);
+  it.p = make_plan(a, lo);
   const int r = idx - prefix[lo];
-  it.kvh = r / p.n_split;
-  it.split = r % p.n_split;
-  const int v0 = it.split * p.chunk;
-  const int v1 = min(p.n_vis, v0 + p.chunk);
-  const int ea = min(v1, p.len0);
-  it.a0 = v0;
-  it.na = max(0, ea - v0);
-  const int sb = max(v0, p.len0);
-  it.b0 = p.lo1 + (sb - p.len0);
-  it.nb = max(0, v1 - sb);
+  it.kvh = r / it.p.n_split;
+  it.split = r % it.p.n_split;
+  it.v0 = it.split * it.p.chunk;
+  it.v1 = min(it.p.n_vis, it.v0 + it.p.chunk);
   return it;
 }
 
+// Stages cover consecutive virtual keys of the item, whatever physical pieces they
+// come from, so a key's stage row (and hence the arithmetic) depends only on its place
+// in the position order: a ring cache and a contiguous cache give identical results.
 __device__ __forceinline__ int item_stages(const Item& it) {
-  return (it.na + kStageKeys - 1) / kStageKeys + (it.nb + kStageKeys - 1) / kStageKeys;
+  return (it.v1 - it.v0 + kStageKeys - 1) / kStageKeys;
 }
 
-// Stage k of an item: first key position and key count.
-__device__ __forceinline__ void item_stage(const Item& it, int k, int& pos, int& n) {
-  const int sa = (it.na + kStageKeys - 1) / kStageKeys;
-  if (k < sa) {
-    pos = it.a0 + k * kStageKeys;
-    n = min(kStageKeys, it.na - k * kStageKeys);
-  } else {
-    const int kk = k - sa;
-    pos = it.b0 + kk * kStageKeys;
-    n = min(kStageKeys, it.nb - kk * kStageKeys);
+__device__ __forceinline__ int stage_keys(const Item& it, int k) {
+  return min(kStageKeys, it.v1 - it.v0 - k * kStageKeys);
+}
+
+// Physical runs of stage k: up to three (first physical row, count, stage row) triples.
+__device__ __forceinline__ int stage_runs(const Item& it, int k, int (&row)[3], int (&cnt)[3],
+                                          int (&dst)[3]) {
+  const int vs = it.v0 + k * kStageKeys;
+  const int ve = min(it.v1, vs + kStageKeys);
+  const int len2 = it.p.n_vis - it.p.len0 - it.p.len1;
+  const int pvs[3] = {0, it.p.len0, it.p.len0 + it.p.len1};
+  const int pln[3] = {it.p.len0, it.p.len1, len2};
+  const int pst[3] = {0, it.p.start1, it.p.start2};
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int a0 = max(vs, pvs[i]);
+    const int a1 = min(ve, pvs[i] + pln[i]);
+    if (a1 > a0) {
+      row[n] = pst[i] + (a0 - pvs[i]);
+      cnt[n] = a1 - a0;
+      dst[n] = a0 - vs;
+      ++n;
+    }
   }
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+  return n;
 }
 
 __device__ __forceinline__ uint4 lds128(const uint16_t* p) {
@@ -257,6 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
     prefix[b + 1] = a.hkv * p.n_split;
     const int T = a.seq_len[b];
     if ((T < 0 || T > a.capacity) && blockIdx.x == 0) atomicOr(a.status, kStatusBadLength);
+    if (a.ring_rows > 0 && T > 0 && blockIdx.x == 0 &&
+        route_is_fa(a.fa_mask, a.mask_words, b, a.layer))
+      atomicOr(a.status, kStatusRingRoute);
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -293,23 +327,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const Item it = item_at(a, prefix, idx);
-        const size_t head_off = (size_t(it.b) * a.hkv + it.kvh) * a.capacity * row_elems;
+        const size_t head_off = (size_t(it.b) * a.hkv + it.kvh) * a.rows * row_elems;
         const uint16_t* qsrc = a.q + (size_t(it.b) * a.hkv * G + size_t(it.kvh) * G) * D;
         const int ns = item_stages(it);
         for (int k = 0; k < ns; ++k, ++g) {
-          int pos, n;
-          item_stage(it, k, pos, n);
+          int row[3], cnt[3], dst[3];
+          const int runs = stage_runs(it, k, row, cnt, dst);
           const int st = g % kStages;
           const uint32_t ph = (g / kStages) & 1;
           if (!mbar_wait(empty0 + 8 * st, ph ^ 1, a.status)) { ok = false; break; }
-          const uint32_t bytes = uint32_t(n) * D * 2;
+          const uint32_t bytes = uint32_t(stage_keys(it, k)) * D * 2;
           const uint32_t qbytes = (k == 0) ? uint32_t(G * D * 2) : 0u;
           mbar_arrive_expect_tx(full0 + 8 * st, 2 * bytes + qbytes);
           if (k == 0) bulk_g2s(smem_addr(sQ + st * L::q_slot), qsrc, qbytes, full0 + 8 * st, pol);
-          bulk_g2s(smem_addr(sK + st * L::kv_stage), a.k + head_off + size_t(pos) * row_elems,
-                   bytes, full0 + 8 * st, pol);
-          bulk_g2s(smem_addr(sV + st * L::kv_stage), a.v + head_off + size_t(pos) * row_elems,
-                   bytes, full0 + 8 * st, pol);
+          for (int r = 0; r < runs; ++r) {
+            const uint32_t rb = uint32_t(cnt[r]) * D * 2;
+            const size_t src = head_off + size_t(row[r]) * row_elems;
+            bulk_g2s(smem_addr(sK + st * L::kv_stage + size_t(dst[r]) * D), a.k + src, rb,
+                     full0 + 8 * st, pol);
+            bulk_g2s(smem_addr(sV + st * L::kv_stage + size_t(dst[r]) * D), a.v + src, rb,
+                     full0 + 8 * st, pol);
+          }
         }
       }
       // never leave the CTA with copies in flight: wait for each stage's last fill
@@ -341,8 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
 
     const int ns = item_stages(it);
     for (int k = 0; k < ns; ++k, ++g) {
-      int pos, n;
-      item_stage(it, k, pos, n);
+      const int n = stage_keys(it, k);
       const int st = g % kStages;
       const uint32_t ph = (g / kStages) & 1;
       if (!mbar_wait(full0 + 8 * st, ph, a.status)) { ok = false; break; }
@@ -399,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
       const float m_new = fmaxf(m_run, mt);
       if (__any_sync(0xffffffffu, m_new > m_run)) {
-        const float alpha = (m_new > m_run) ? fast_exp2(m_run - m_new) : 1.f;
+        const float alpha = (m_new > m_run) ? ex2_mufu(m_run - m_new) : 1.f;
         l_run *= alpha;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -414,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       float* Pw = sP + warp * kKeysPerWarp * G;
 #pragma unroll
       for (int p = 0; p < kPasses; ++p) {
-        const float pr = fast_exp2(s[p] - m_use);
+        const float pr = ex2_mufu(s[p] - m_use);
         l_run += pr;
         if (owner) Pw[(p * 4 + key_sub) * G + hl] = pr;
       }
@@ -492,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
         const float mw = sM[w * G + h];
-        const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+        const float f = (mw == -INFINITY) ? 0.f : ex2_mufu(mw - M);
         av = fmaf(f, sAcc[(w * G + h) * D + e], av);
         lv = fmaf(f, sL[w * G + h], lv);
       }
@@ -528,8 +565,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a)
     float M = fmaxf(m0, m1);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float f0 = (lane < p.n_split) ? fast_exp2(m0 - M) : 0.f;
-    const float f1 = (lane + 32 < p.n_split) ? fast_exp2(m1 - M) : 0.f;
+    const float f0 = (lane < p.n_split) ? ex2_mufu(m0 - M) : 0.f;
+    const float f1 = (lane + 32 < p.n_split) ? ex2_mufu(m1 - M) : 0.f;
     float lv = f0 * l0 + f1 * l1;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, off);
@@ -615,8 +652,8 @@ size_t decode_workspace_bytes(const AttnGeom& g, int batch) {
 
 cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
-                          const int32_t* seq_len, int batch, int capacity, uint16_t* o,
-                          void* workspace, unsigned* status, cudaStream_t stream) {
+                          const int32_t* seq_len, int batch, int capacity, int ring_rows,
+                          uint16_t* o, void* workspace, unsigned* status, cudaStream_t stream) {
   const int G = g.hq / g.hkv;
   DecodeArgs a;
   a.fa_mask = fa_mask;
@@ -627,7 +664,9 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
   a.v = v_cache;
   a.seq_len = seq_len;
   a.batch = batch;
-  a.capacity = capacity;
+  a.ring_rows = ring_rows;
+  a.rows = ring_rows > 0 ? g.sink + ring_rows : capacity;
+  a.capacity = ring_rows > 0 ? 0x7fffffff : capacity;  // a ring never runs out of rows
   a.hkv = g.hkv;
   a.block = g.block;
   a.sink = g.sink;
@@ -667,7 +706,7 @@ cudaError_t launch_decode_static(const AttnGeom& g, int layer, const uint32_t* f
   void* scratch = nullptr;
   const cudaError_t err = static_scratch_address(&scratch);
   if (err != cudaSuccess) return err;
-  return launch_decode(g, layer, fa_mask, q, k_cache, v_cache, seq_len, batch, capacity, o,
+  return launch_decode(g, layer, fa_mask, q, k_cache, v_cache, seq_len, batch, capacity, 0, o,
                        scratch, status, stream);
 }
 

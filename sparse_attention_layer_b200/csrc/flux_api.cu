@@ -216,7 +216,7 @@ int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask
   unsigned* status = flux::status_ptr();
   if (!status) return FLUX_ERR_CUDA;
   return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_cache, v_cache, seq_len,
-                                               batch, capacity, o, workspace, status,
+                                               batch, capacity, 0, o, workspace, status,
                                                static_cast<cudaStream_t>(stream)));
 }
 
@@ -238,6 +238,64 @@ int flux_decode_static(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* 
   return flux::cuda_status(flux::launch_decode_static(g, layer, fa_mask, q, k_cache, v_cache,
                                                       seq_len, batch, capacity, o, status,
                                                       static_cast<cudaStream_t>(stream)));
+}
+
+int flux_kv_compact_ring(const flux_attn_cfg* cfg, const uint16_t* k_cache,
+                         const uint16_t* v_cache, int32_t capacity, const int32_t* seq_len,
+                         int32_t batch, uint16_t* k_ring, uint16_t* v_ring, int32_t ring_rows,
+                         void* stream) {
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!k_cache || !v_cache || !seq_len || !k_ring || !v_ring) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || capacity < 1) return FLUX_ERR_INVALID_ARG;
+  if (ring_rows < cfg->window) return FLUX_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_ring) || !aligned16(v_ring))
+    return FLUX_ERR_INVALID_ARG;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  return flux::cuda_status(flux::launch_kv_compact_ring(flux::geom_of(cfg), k_cache, v_cache,
+                                                        capacity, seq_len, batch, k_ring, v_ring,
+                                                        ring_rows, status,
+                                                        static_cast<cudaStream_t>(stream)));
+}
+
+int flux_kv_append_ring(const flux_attn_cfg* cfg, uint16_t* k_ring, uint16_t* v_ring,
+                        int32_t* seq_len, int32_t batch, int32_t ring_rows,
+                        const uint16_t* k_new, const uint16_t* v_new, int32_t n_new,
+                        void* stream) {
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!k_ring || !v_ring || !seq_len || !k_new || !v_new) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || n_new < 0) return FLUX_ERR_INVALID_ARG;
+  if (ring_rows < cfg->window || n_new > ring_rows) return FLUX_ERR_INVALID_ARG;
+  if (!aligned16(k_ring) || !aligned16(v_ring) || !aligned16(k_new) || !aligned16(v_new))
+    return FLUX_ERR_INVALID_ARG;
+  if (n_new == 0) return FLUX_OK;
+  return flux::cuda_status(flux::launch_kv_append_ring(flux::geom_of(cfg), k_ring, v_ring,
+                                                       seq_len, batch, ring_rows, k_new, v_new,
+                                                       n_new, static_cast<cudaStream_t>(stream)));
+}
+
+int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                     const uint16_t* q, const uint16_t* k_ring, const uint16_t* v_ring,
+                     const int32_t* seq_len, int32_t batch, int32_t ring_rows, uint16_t* o,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!fa_mask || !q || !k_ring || !v_ring || !seq_len || !o) return FLUX_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= cfg->n_layers) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > flux::kDecMaxBatch) return FLUX_ERR_INVALID_ARG;
+  if (ring_rows < cfg->window) return FLUX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring)) return FLUX_ERR_INVALID_ARG;
+  const flux::AttnGeom g = flux::geom_of(cfg);
+  if (!workspace || workspace_bytes < flux::decode_workspace_bytes(g, batch) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return FLUX_ERR_WORKSPACE;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_ring, v_ring, seq_len,
+                                               batch, 0, ring_rows, o, workspace, status,
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 int flux_sa_block_ranges(const flux_attn_cfg* cfg, int32_t n_qblocks, int32_t* ranges,

@@ -18,6 +18,7 @@ namespace flux {
 constexpr unsigned kStatusCapacity = 0x1u;
 constexpr unsigned kStatusTimeout = 0x2u;
 constexpr unsigned kStatusBadLength = 0x4u;
+constexpr unsigned kStatusRingRoute = 0x8u;
 
 // A pipeline wait gives up after this long (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -20,10 +20,12 @@ constexpr int kDecMaxBatch = 1024;
 
 size_t decode_workspace_bytes(const AttnGeom& g, int batch);
 
+// ring_rows == 0: contiguous cache of `capacity` rows per (sequence, KV head);
+// ring_rows > 0: SA ring cache of sink + ring_rows rows (capacity unused).
 cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
-                          const int32_t* seq_len, int batch, int capacity, uint16_t* o,
-                          void* workspace, unsigned* status, cudaStream_t stream);
+                          const int32_t* seq_len, int batch, int capacity, int ring_rows,
+                          uint16_t* o, void* workspace, unsigned* status, cudaStream_t stream);
 
 // Decode with the library's own file-scope scratch array instead of a caller
 // workspace (flux_decode_static).  Its size is FLUX_DECODE_STATIC_SCRATCH_BYTES.
@@ -38,6 +40,16 @@ cudaError_t launch_kv_append(const AttnGeom& g, uint16_t* k_cache, uint16_t* v_c
                              int32_t* seq_len, int batch, int capacity, const uint16_t* k_new,
                              const uint16_t* v_new, int n_new, unsigned* status,
                              cudaStream_t stream);
+
+// SA ring caches: compaction from a full cache, and append
+cudaError_t launch_kv_compact_ring(const AttnGeom& g, const uint16_t* k_cache,
+                                   const uint16_t* v_cache, int capacity, const int32_t* seq_len,
+                                   int batch, uint16_t* k_ring, uint16_t* v_ring, int ring_rows,
+                                   unsigned* status, cudaStream_t stream);
+cudaError_t launch_kv_append_ring(const AttnGeom& g, uint16_t* k_ring, uint16_t* v_ring,
+                                  int32_t* seq_len, int batch, int ring_rows,
+                                  const uint16_t* k_new, const uint16_t* v_new, int n_new,
+                                  cudaStream_t stream);
 
 // ----- router
 constexpr int kRouterMaxHidden = 16384;

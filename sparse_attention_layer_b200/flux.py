@@ -28,12 +28,14 @@ FLUX_ERR_WORKSPACE = 6
 FLUX_DEVICE_CAPACITY = 0x1
 FLUX_DEVICE_TIMEOUT = 0x2
 FLUX_DEVICE_BAD_LENGTH = 0x4
+FLUX_DEVICE_RING_ROUTE = 0x8
 
 # every entry point declared in include/flux.h
 EXPORTED = (
     "flux_mask_words", "flux_route", "flux_kv_append", "flux_prefill",
     "flux_decode_workspace_size", "flux_decode", "flux_sa_block_ranges",
     "flux_get_device_status", "flux_status_string", "flux_version", "flux_decode_static",
+    "flux_kv_compact_ring", "flux_kv_append_ring", "flux_decode_ring",
 )
 
 # bytes of the scratch array flux_decode_static keeps inside the library
@@ -121,6 +123,15 @@ def lib() -> ctypes.CDLL:
         L.flux_decode_static.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32,
                                          i32, vp, vp]
         L.flux_decode_static.restype = ctypes.c_int
+        L.flux_kv_compact_ring.argtypes = [ctypes.POINTER(FluxAttnCfg), vp, vp, i32, vp, i32, vp,
+                                           vp, i32, vp]
+        L.flux_kv_compact_ring.restype = ctypes.c_int
+        L.flux_kv_append_ring.argtypes = [ctypes.POINTER(FluxAttnCfg), vp, vp, vp, i32, i32, vp,
+                                          vp, i32, vp]
+        L.flux_kv_append_ring.restype = ctypes.c_int
+        L.flux_decode_ring.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32,
+                                       i32, vp, vp, sz, vp]
+        L.flux_decode_ring.restype = ctypes.c_int
         L.flux_sa_block_ranges.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp]
         L.flux_sa_block_ranges.restype = ctypes.c_int
         _lib = L
@@ -273,6 +284,55 @@ def flux_decode_static(cfg: AttnCfg, layer: int, fa_mask, q, k_cache, v_cache, s
         _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, cap,
         _ptr(o, "o", torch.bfloat16, (batch, hq, d)), _stream(stream))
     _check("flux_decode_static", st)
+
+
+def flux_kv_compact_ring(cfg: AttnCfg, k_cache, v_cache, seq_len, k_ring, v_ring,
+                         stream=None) -> None:
+    """Copy the rows an SA layer still needs from a full cache [B][Hkv][cap][d] into
+    ring caches [B][Hkv][sink + ring_rows][d]."""
+    batch, hkv, cap, d = k_cache.shape
+    rows = k_ring.shape[2]
+    c = cfg.c()
+    st = lib().flux_kv_compact_ring(
+        ctypes.byref(c), _ptr(k_cache, "k_cache", torch.bfloat16, (batch, hkv, cap, d)),
+        _ptr(v_cache, "v_cache", torch.bfloat16, (batch, hkv, cap, d)), cap,
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch,
+        _ptr(k_ring, "k_ring", torch.bfloat16, (batch, hkv, rows, d)),
+        _ptr(v_ring, "v_ring", torch.bfloat16, (batch, hkv, rows, d)), rows - cfg.sink,
+        _stream(stream))
+    _check("flux_kv_compact_ring", st)
+
+
+def flux_kv_append_ring(cfg: AttnCfg, k_ring, v_ring, seq_len, k_new, v_new,
+                        stream=None) -> None:
+    """Append k_new/v_new [B][n][Hkv][d] to ring caches and advance seq_len."""
+    batch, hkv, rows, d = k_ring.shape
+    n_new = k_new.shape[1]
+    c = cfg.c()
+    st = lib().flux_kv_append_ring(
+        ctypes.byref(c), _ptr(k_ring, "k_ring", torch.bfloat16, (batch, hkv, rows, d)),
+        _ptr(v_ring, "v_ring", torch.bfloat16, (batch, hkv, rows, d)),
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, rows - cfg.sink,
+        _ptr(k_new, "k_new", torch.bfloat16, (batch, n_new, hkv, d)),
+        _ptr(v_new, "v_new", torch.bfloat16, (batch, n_new, hkv, d)), n_new, _stream(stream))
+    _check("flux_kv_append_ring", st)
+
+
+def flux_decode_ring(cfg: AttnCfg, layer: int, fa_mask, q, k_ring, v_ring, seq_len, o,
+                     workspace, stream=None) -> None:
+    """flux_decode of an SA layer whose cache was compacted into a ring."""
+    batch, hq, d = q.shape
+    rows = k_ring.shape[2]
+    c = cfg.c()
+    st = lib().flux_decode_ring(
+        ctypes.byref(c), int(layer), _ptr(fa_mask, "fa_mask", torch.int32, (batch, cfg.mask_words)),
+        _ptr(q, "q", torch.bfloat16), _ptr(k_ring, "k_ring", torch.bfloat16,
+                                           (batch, cfg.n_kv_heads, rows, d)),
+        _ptr(v_ring, "v_ring", torch.bfloat16, (batch, cfg.n_kv_heads, rows, d)),
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, rows - cfg.sink,
+        _ptr(o, "o", torch.bfloat16, (batch, hq, d)),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("flux_decode_ring", st)
 
 
 def flux_sa_block_ranges(cfg: AttnCfg, n_qblocks: int, ranges, stream=None) -> None:

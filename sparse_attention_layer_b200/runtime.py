@@ -26,6 +26,24 @@ class LayerCache:
             self.seq_len.copy_(torch.as_tensor(lengths, dtype=torch.int32))
 
 
+class RingCache:
+    """An SA layer's decode-time cache after eviction: sink rows plus a ring of
+    ring_rows recent rows ([B][Hkv][sink + ring_rows][d]); seq_len counts positions."""
+
+    def __init__(self, cfg: AttnCfg, batch: int, ring_rows: int, device):
+        shape = (batch, cfg.n_kv_heads, cfg.sink + ring_rows, cfg.head_dim)
+        self.k = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.v = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.seq_len = torch.zeros(batch, dtype=torch.int32, device=device)
+        self.ring_rows = ring_rows
+
+    def reset(self, lengths=None):
+        if lengths is None:
+            self.seq_len.zero_()
+        else:
+            self.seq_len.copy_(torch.as_tensor(lengths, dtype=torch.int32))
+
+
 class HybridAttention:
     """Router + per-layer FA/SA attention over per-layer KV caches."""
 
@@ -53,9 +71,46 @@ class HybridAttention:
 
     def decode_layer(self, layer: int, q, k_new, v_new, out, cache_index=None):
         c = self.caches[layer if cache_index is None else cache_index]
+        if isinstance(c, RingCache):
+            flux.flux_kv_append_ring(self.cfg, c.k, c.v, c.seq_len, k_new, v_new)
+            flux.flux_decode_ring(self.cfg, layer, self.fa_mask, q, c.k, c.v, c.seq_len, out,
+                                  self.workspace)
+            return
         flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, k_new, v_new)
         flux.flux_decode(self.cfg, layer, self.fa_mask, q, c.k, c.v, c.seq_len, out,
                          self.workspace)
+
+    def sa_layers(self) -> list:
+        """Layers every sequence routes to SA (reads the mask once, after routing:
+        routing is decided at prefill and reused by every decode step)."""
+        words = self.fa_mask.cpu()
+        out = []
+        for layer in range(self.cfg.n_layers):
+            bits = [(int(words[b, layer // 32]) >> (layer % 32)) & 1 for b in range(self.batch)]
+            if not any(bits):
+                out.append(layer)
+        return out
+
+    def evict_sa_layers(self, ring_rows: int = 0) -> int:
+        """After prefill: move the cache of every all-SA layer into a ring cache of
+        sink + ring_rows rows (ring_rows defaults to the window) and free the full
+        cache.  Returns the bytes of KV cache freed."""
+        ring_rows = ring_rows or self.cfg.window
+        freed = 0
+        for layer in self.sa_layers():
+            full = self.caches[layer]
+            if isinstance(full, RingCache):
+                continue
+            ring = RingCache(self.cfg, self.batch, ring_rows, self.device)
+            flux.flux_kv_compact_ring(self.cfg, full.k, full.v, full.seq_len, ring.k, ring.v)
+            ring.seq_len.copy_(full.seq_len)
+            freed += (full.k.numel() + full.v.numel() - ring.k.numel() - ring.v.numel()) * 2
+            self.caches[layer] = ring
+        return freed
+
+    def kv_bytes(self) -> int:
+        """Bytes of KV cache currently held (K and V of every layer)."""
+        return sum((c.k.numel() + c.v.numel()) * 2 for c in self.caches)
 
 
 class DecodeStepGraph:

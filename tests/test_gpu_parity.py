@@ -353,3 +353,113 @@ def test_decode_graph_replay_matches_eager():
         torch.cuda.synchronize()
         assert torch.equal(o, o_e), f"step {step}"
     assert [int(c.seq_len[0]) for c in graph_m.caches] == [ctx + steps] * 3
+
+
+# ------------------------------------------------------ SA ring caches (KV eviction)
+
+
+def _ring_setup(cfg, ctx, ring_rows, seed):
+    case = CacheCase(cfg, ctx, max(ctx) + 200, seed)
+    rows = cfg.sink + ring_rows
+    k_ring = torch.zeros(len(ctx), cfg.n_kv_heads, rows, cfg.head_dim, dtype=torch.bfloat16,
+                         device="cuda")
+    v_ring = torch.zeros_like(k_ring)
+    flux.flux_kv_compact_ring(cfg, case.k, case.v, case.seq_len, k_ring, v_ring)
+    ring_len = case.seq_len.clone()
+    return case, k_ring, v_ring, ring_len
+
+
+def _retained_equal(cfg, ring_rows, k_ring, full_host, lens):
+    for b, T in enumerate(lens):
+        pos = orc.ring_retained_positions(int(T), cfg.sink, ring_rows)
+        slots = orc.ring_slot(pos, cfg.sink, ring_rows)
+        got = k_ring[b][:, torch.as_tensor(slots)].cpu().view(torch.int16)
+        want = full_host[b][:, torch.as_tensor(pos)].view(torch.int16)
+        assert torch.equal(got, want), (b, T)
+
+
+def test_ring_compact_and_append_exact():
+    cfg = AttnCfg(1, 8, 2, 128, 64, 128, 256)
+    ring_rows = 320
+    ctx = [0, 50, 128, 300, 449, 450, 1000, 1777]
+    case, k_ring, v_ring, ring_len = _ring_setup(cfg, ctx, ring_rows, seed=5)
+    _retained_equal(cfg, ring_rows, k_ring, case.k_host, ctx)
+    _retained_equal(cfg, ring_rows, v_ring, case.v_host, ctx)
+    for step in range(3):
+        kn = inputs.normal_bf16((len(ctx), 1, 2, 128), 300 + step)
+        vn = inputs.normal_bf16((len(ctx), 1, 2, 128), 400 + step)
+        flux.flux_kv_append_ring(cfg, k_ring, v_ring, ring_len, kn.cuda(), vn.cuda())
+        case.append(kn, vn)
+    lens = case.seq_len.cpu().tolist()
+    assert ring_len.cpu().tolist() == lens
+    _retained_equal(cfg, ring_rows, k_ring, case.k_host, lens)
+    _retained_equal(cfg, ring_rows, v_ring, case.v_host, lens)
+    assert flux.flux_get_device_status() == 0
+
+
+@pytest.mark.parametrize("block,sink,window,ring_extra", [(64, 64, 256, 0), (128, 128, 512, 64),
+                                                          (64, 0, 128, 0)])
+def test_ring_decode_identical_to_full(block, sink, window, ring_extra):
+    """Decode over the ring equals decode over the full cache bit for bit (same keys,
+    same split plan) and the oracle within tolerance, across the ring's wrap-around."""
+    cfg = AttnCfg(1, 8, 2, 128, block, sink, window)
+    ring_rows = window + ring_extra
+    ctx = [1, sink + 3, sink + window - 1, sink + window + 1, 3 * window + 17, 4000]
+    case, k_ring, v_ring, ring_len = _ring_setup(cfg, ctx, ring_rows, seed=9)
+    batch = len(ctx)
+    mask = mask_words(batch, 1, [[] for _ in ctx]).cuda()
+    ws = torch.empty(flux.flux_decode_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    for step in range(block + 3):   # crosses a block boundary and wraps the ring
+        kn = inputs.normal_bf16((batch, 1, 2, 128), 500 + step)
+        vn = inputs.normal_bf16((batch, 1, 2, 128), 600 + step)
+        q = inputs.normal_bf16((batch, 8, 128), 700 + step).cuda()
+        case.append(kn, vn)
+        flux.flux_kv_append_ring(cfg, k_ring, v_ring, ring_len, kn.cuda(), vn.cuda())
+        o_full = torch.empty(batch, 8, 128, dtype=torch.bfloat16, device="cuda")
+        o_ring = torch.empty_like(o_full)
+        flux.flux_decode(cfg, 0, mask, q, case.k, case.v, case.seq_len, o_full, ws)
+        flux.flux_decode_ring(cfg, 0, mask, q, k_ring, v_ring, ring_len, o_ring, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(o_ring, o_full), f"step {step}"
+        if step % 16 == 0:
+            want = oracle_layer(case, q.cpu()[:, None], [False] * batch)[:, 0]
+            assert_close(f64(o_ring), want, f"ring decode step {step}")
+    assert flux.flux_get_device_status() == 0
+
+
+def test_ring_decode_refuses_fa_route():
+    cfg = AttnCfg(1, 4, 1, 64, 64, 64, 64)
+    k = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
+    seq = torch.tensor([100], dtype=torch.int32, device="cuda")
+    mask = torch.ones(1, 1, dtype=torch.int32, device="cuda")  # layer 0 routed to FA
+    ws = torch.empty(flux.flux_decode_workspace_size(cfg, 1), dtype=torch.uint8, device="cuda")
+    o = torch.full((1, 4, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    flux.flux_decode_ring(cfg, 0, mask, torch.ones_like(o), k, k, seq, o, ws)
+    assert flux.flux_get_device_status() & flux.FLUX_DEVICE_RING_ROUTE
+    assert (o == 0).all()
+
+
+def test_ring_decode_llama_full_size():
+    """Llama-3.1-8B decode shape: 16 sequences at 32K context, an SA layer evicted to a
+    2048-row ring (2176 rows per head instead of 33024): identical to the full cache."""
+    w = configs.LLAMA_DECODE
+    cfg = cfg_of(w)
+    ctx = [w.seq] * w.batch
+    case, k_ring, v_ring, ring_len = _ring_setup(cfg, ctx, w.window, seed=1002)
+    mask = mask_words(w.batch, cfg.n_layers, [[] for _ in ctx]).cuda()
+    ws = torch.empty(flux.flux_decode_workspace_size(cfg, w.batch), dtype=torch.uint8,
+                     device="cuda")
+    for step in range(2):
+        kn = inputs.normal_bf16((w.batch, 1, 8, 128), 800 + step)
+        vn = inputs.normal_bf16((w.batch, 1, 8, 128), 900 + step)
+        q = inputs.normal_bf16((w.batch, 32, 128), 1000 + step).cuda()
+        case.append(kn, vn)
+        flux.flux_kv_append_ring(cfg, k_ring, v_ring, ring_len, kn.cuda(), vn.cuda())
+        o_full = torch.empty(w.batch, 32, 128, dtype=torch.bfloat16, device="cuda")
+        o_ring = torch.empty_like(o_full)
+        flux.flux_decode(cfg, 7, mask, q, case.k, case.v, case.seq_len, o_full, ws)
+        flux.flux_decode_ring(cfg, 7, mask, q, k_ring, v_ring, ring_len, o_ring, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(o_ring, o_full)
+    want = oracle_layer(case, q.cpu()[:, None], [False] * w.batch)[:, 0]
+    assert_close(f64(o_ring), want, "ring decode at 32K")
