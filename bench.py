@@ -537,7 +537,51 @@ def run_flux(args, world, rank, local):
     for v in mix.values():
         v["speedup_vs_all_fa"] = base / v["ms_per_step"]
     db.set_sa_layers(db.sa_layers)
-    del graph, db
+    del graph
+
+    # ---------------- SA-layer KV eviction: rings of sink + window rows per SA layer
+    db.reset()
+    kv_full = db.model.kv_bytes()
+    freed = db.model.evict_sa_layers()
+    torch.cuda.synchronize()
+    kv_evicted = db.model.kv_bytes()
+    db.reset()
+    for c in db.model.caches:
+        c.seq_len.fill_(db.ctx)
+    ring_graph = DecodeStepGraph(db.model, db.q, db.k_new, db.v_new, db.o)
+    for c in db.model.caches:
+        c.seq_len.fill_(db.ctx)
+    for _ in range(args.warmup):
+        ring_graph.replay()
+    for c in db.model.caches:
+        c.seq_len.fill_(db.ctx)
+    barrier(world)
+    rs = torch.cuda.Event(enable_timing=True)
+    re_ = torch.cuda.Event(enable_timing=True)
+    rs.record()
+    for _ in range(args.steps):
+        ring_graph.replay()
+    re_.record()
+    barrier(world)
+    tr_ms = max_over_ranks(rs.elapsed_time(re_), world)
+    st = flux.flux_get_device_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} after the ring decode steps")
+    gib = float(1 << 30)
+    per_seq_full = kv_full / w.batch
+    per_seq_evicted = kv_evicted / w.batch
+    hbm_budget = 160 * gib  # leaves room for weights and activations on a 180 GB part
+    eviction = {
+        "kv_gib_full": kv_full / gib, "kv_gib_evicted": kv_evicted / gib,
+        "saving": 1.0 - kv_evicted / kv_full,
+        "decode_tokens_per_s": replica_tokens_per_s(world, w.batch, args.steps, tr_ms),
+        "ms_per_step": tr_ms / args.steps,
+        "max_batch_in_160_gib": {"full": int(hbm_budget // per_seq_full),
+                                 "evicted": int(hbm_budget // per_seq_evicted)},
+        "what": "the 16 SA layers' caches moved to rings of sink 128 + 2048 rows per "
+                "(sequence, KV head) after prefill; the same graph-replayed decode step",
+    }
+    del ring_graph, db
     torch.cuda.empty_cache()
 
     # ---------------- prefill phase (Llama shape, 8192 tokens, router-chosen routes)
@@ -601,7 +645,7 @@ def run_flux(args, world, rank, local):
                         "fa_layer_bytes": fa_bytes, "sa_layer_bytes": sa_bytes},
         "cpu_baseline": cpu, "e2e": e2e, "decode_eager": eager,
         "gpu_launches": w.n_layers * 4 * args.steps, "clocks": clocks,
-        "prefill": prefill, "routing_mix": mix,
+        "prefill": prefill, "routing_mix": mix, "sa_kv_eviction": eviction,
     }
     if rank == 0:
         print(json.dumps(line))
