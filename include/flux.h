@@ -231,6 +231,13 @@ int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa
 int flux_sa_block_ranges(const flux_attn_cfg* cfg, int32_t n_qblocks, int32_t* ranges,
                          void* stream);
 
+/* flux_selftest_wait_timeout -- failure-detection self-test (the paper has no
+ * counterpart): one thread waits on an mbarrier that nothing releases, through the
+ * bounded wait every pipeline wait of the library uses, with a limit of limit_us
+ * microseconds (1..1000000).  The wait gives up, FLUX_DEVICE_TIMEOUT is set in the
+ * device status word and the kernel returns; the context stays usable. */
+int flux_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Copy the device status word of the current device to *bits and clear it.
  * Synchronises `stream` first. */
 int flux_get_device_status(void* stream, uint32_t* bits);

@@ -52,6 +52,17 @@ __global__ void sa_block_ranges_kernel(int n_qblocks, int n_sink_blocks, int n_w
   ranges[3 * qb + 2] = r.win_end;
 }
 
+// One thread waits on an mbarrier that nothing arrives on, through the same bounded
+// wait every pipeline wait in the library uses.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  mbar_wait(b, 0, status, limit_ns);
+}
+
 int validate_cfg(const flux_attn_cfg* c) {
   if (!c) return FLUX_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->n_layers > 1024) return FLUX_ERR_INVALID_ARG;
@@ -125,6 +136,15 @@ const char* flux_status_string(int status) {
     case FLUX_ERR_WORKSPACE: return "workspace missing or too small";
     default: return "unknown status";
   }
+}
+
+int flux_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return FLUX_ERR_INVALID_ARG;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  flux::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_us * 1000ull, status);
+  return flux::cuda_status(cudaGetLastError());
 }
 
 int flux_get_device_status(void* stream, uint32_t* bits) {

@@ -201,8 +201,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and sets
-// the timeout bit) if it does not within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status) {
+// the timeout bit) if it does not within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
 #pragma unroll 1
   for (int i = 0; i < 16; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -210,7 +211,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 #pragma unroll 1
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       atomicOr(status, kStatusTimeout);
       return false;
     }

@@ -36,6 +36,7 @@ EXPORTED = (
     "flux_decode_workspace_size", "flux_decode", "flux_sa_block_ranges",
     "flux_get_device_status", "flux_status_string", "flux_version", "flux_decode_static",
     "flux_kv_compact_ring", "flux_kv_append_ring", "flux_decode_ring",
+    "flux_selftest_wait_timeout",
 )
 
 # bytes of the scratch array flux_decode_static keeps inside the library
@@ -132,6 +133,8 @@ def lib() -> ctypes.CDLL:
         L.flux_decode_ring.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32,
                                        i32, vp, vp, sz, vp]
         L.flux_decode_ring.restype = ctypes.c_int
+        L.flux_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
+        L.flux_selftest_wait_timeout.restype = ctypes.c_int
         L.flux_sa_block_ranges.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp]
         L.flux_sa_block_ranges.restype = ctypes.c_int
         _lib = L
@@ -333,6 +336,12 @@ def flux_decode_ring(cfg: AttnCfg, layer: int, fa_mask, q, k_ring, v_ring, seq_l
         _ptr(o, "o", torch.bfloat16, (batch, hq, d)),
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check("flux_decode_ring", st)
+
+
+def flux_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Launch a wait that nothing releases; it must time out into FLUX_DEVICE_TIMEOUT."""
+    _check("flux_selftest_wait_timeout",
+           lib().flux_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def flux_sa_block_ranges(cfg: AttnCfg, n_qblocks: int, ranges, stream=None) -> None:

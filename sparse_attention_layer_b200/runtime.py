@@ -69,6 +69,24 @@ class HybridAttention:
         flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, k_new, v_new)
         flux.flux_prefill(self.cfg, layer, self.fa_mask, q, c.k, c.v, c.seq_len, out)
 
+    def prefill_layer_chunked(self, layer: int, q, k_new, v_new, out, chunk: int = 16384):
+        """Prefill a long prompt in chunks of `chunk` tokens (Table 6 of the paper page
+        runs its SA kernel with chunk 16384): each chunk appends its K/V rows, then its
+        queries attend everything before them.  With chunk a multiple of 128 the
+        result equals a one-shot prefill bit for bit (same tiles, same order).
+        q/out [B][S][Hq][d], k_new/v_new [B][S][Hkv][d]."""
+        c = self.caches[layer]
+        seq = q.shape[1]
+        for c0 in range(0, seq, chunk):
+            c1 = min(seq, c0 + chunk)
+            qc = q[:, c0:c1].contiguous()
+            oc = out[:, c0:c1] if q.shape[0] == 1 else torch.empty_like(qc)
+            flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, k_new[:, c0:c1].contiguous(),
+                                v_new[:, c0:c1].contiguous())
+            flux.flux_prefill(self.cfg, layer, self.fa_mask, qc, c.k, c.v, c.seq_len, oc)
+            if q.shape[0] != 1:
+                out[:, c0:c1].copy_(oc)
+
     def decode_layer(self, layer: int, q, k_new, v_new, out, cache_index=None):
         c = self.caches[layer if cache_index is None else cache_index]
         if isinstance(c, RingCache):

@@ -463,3 +463,60 @@ def test_ring_decode_llama_full_size():
         assert torch.equal(o_ring, o_full)
     want = oracle_layer(case, q.cpu()[:, None], [False] * w.batch)[:, 0]
     assert_close(f64(o_ring), want, "ring decode at 32K")
+
+
+# --------------------------------------------------------- failure detection, chunks
+
+
+def test_wait_timeout_selftest_reports_and_recovers():
+    """A pipeline wait that nothing releases gives up after its limit, reports
+    FLUX_DEVICE_TIMEOUT through the status word, and the context keeps working."""
+    flux.flux_selftest_wait_timeout(2000)
+    assert flux.flux_get_device_status() & flux.FLUX_DEVICE_TIMEOUT
+    assert flux.flux_get_device_status() == 0  # read-and-clear
+    cfg = AttnCfg(1, 4, 1, 64, 64, 64, 128)
+    _decode_case(cfg, [300], [False], 1, seed=77)
+
+
+@pytest.mark.parametrize("fa", [True, False])
+def test_chunked_prefill_identical_to_one_shot(fa):
+    """Qwen3-4B shape, 40000-token prompt in 16384-token chunks (Table 6's chunk size):
+    bit-identical to the one-shot prefill, and within tolerance of the oracle."""
+    from sparse_attention_layer_b200.runtime import HybridAttention
+    w = configs.QWEN_PREFILL
+    cfg = AttnCfg(1, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.sink, w.window)
+    S = 40000
+    q = inputs.normal_bf16((1, S, 32, 128), 1).cuda()
+    k = inputs.normal_bf16((1, S, 8, 128), 2).cuda()
+    v = inputs.normal_bf16((1, S, 8, 128), 3).cuda()
+    mask = mask_words(1, 1, [[0] if fa else []]).cuda()
+    outs = []
+    for chunk in (None, 16384):
+        m = HybridAttention(cfg, 1, S, "cuda")
+        m.set_mask(mask)
+        o = torch.empty_like(q)
+        if chunk is None:
+            m.prefill_layer(0, q, k, v, o)
+        else:
+            m.prefill_layer_chunked(0, q, k, v, o, chunk=chunk)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
+    rows = np.array([0, 16383, 16384, 16385, 32767, 32768, S - 1, 20000])
+    kc = k.cpu()[0].transpose(0, 1).float().numpy().astype(np.float64)[None]
+    vc = v.cpu()[0].transpose(0, 1).float().numpy().astype(np.float64)[None]
+    want = orc.attention_layer(q.cpu().float().numpy().astype(np.float64), kc, vc,
+                               np.array([S]), np.array([fa]), cfg.block, cfg.sink, cfg.window,
+                               rows=rows, heads=[0, 13])
+    got = outs[1].cpu()[:, torch.as_tensor(rows)][:, :, torch.as_tensor([0, 13])]
+    assert_close(f64(got), want, "chunked prefill")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("fa", [True, False])
+def test_prefill_pages_sa_geometry(d, fa):
+    """The pages' SA kernel geometry (Table 6): block 64, sink 128, with a 2048-token
+    window, Llama heads, head_dim 64 and 128; sampled rows of a 6000-token prompt."""
+    cfg = AttnCfg(1, 32, 8, d, 64, 128, 2048)
+    rows = sample_rows(6000, 0, cfg, 24, seed=3)
+    _prefill_case(cfg, [0], 6000, [fa], seed=1100 + d + fa, rows=rows, heads=[0, 9, 31])

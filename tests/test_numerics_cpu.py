@@ -24,7 +24,7 @@ def exp2_poly(x):
 
 
 def test_poly_exp2_relative_error():
-    x = np.linspace(-125.0, 8.0, 2_000_001).astype(np.float32)
+    x = np.linspace(-125.0, 8.0, 400_001).astype(np.float32)
     got = exp2_poly(x).astype(np.float64)
     want = np.exp2(x.astype(np.float64))
     rel = np.abs(got / want - 1.0)
