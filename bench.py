@@ -652,6 +652,125 @@ def run_flux(args, world, rank, local):
 
 
 
+def run_sweep(args):
+    """Routing-mix x context x batch sweep of the Llama-3.1-8B shape (32 layers, 32/8
+    heads, d 128, sink 128 + window 2048, block 128).  Every point is a measured
+    32-layer step replayed from a CUDA graph with the given fraction of layers routed to
+    SA (a fixed seeded choice of layers):
+      decode  -- KV append + FA/SA decode per layer; the layers cycle over n distinct
+                 KV caches, n = 32 where they fit in 120 GB and at least 512 MB of
+                 cache is read between two visits of the same cache (so repeated
+                 layers are not served from L2);
+      prefill -- batch 1, KV append + FA/SA prefill on 32 separate caches.
+    Per-layer FA and SA times are the 0 % and 100 % steps divided by 32."""
+    from sparse_attention_layer_b200 import configs, inputs
+    from sparse_attention_layer_b200.flux import AttnCfg
+    from sparse_attention_layer_b200.runtime import HybridAttention
+    torch.cuda.set_device(0)
+    n_layers = 32
+    cfg = AttnCfg(n_layers, 32, 8, 128, 128, 128, 2048)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    fracs = configs.SWEEP_SA_FRACTIONS
+    out = {"decode": [], "prefill": []}
+
+    def graph_ms(graph, warm, reps):
+        for _ in range(warm):
+            graph.replay()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for a, b in ev:
+            a.record(); graph.replay(); b.record()
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    def mask_for(model, batch, frac):
+        sa = inputs.fixed_sa_layers(n_layers, int(round(frac * n_layers)), seed=11)
+        model.set_mask(inputs.pack_bits_u32(inputs.fa_bits_from_sa_layers(batch, n_layers, sa)).cuda())
+
+    warm, reps = 3, 10
+    sampler = ClockSampler(0)
+    sampler.start()
+    for T in configs.SWEEP_CONTEXTS:
+        for B in configs.SWEEP_BATCHES:
+            cap = T + n_layers * (warm + reps + 1) + 64
+            cache_bytes = 2 * B * cfg.n_kv_heads * cap * cfg.head_dim * 2
+            n_cache = max(1, min(n_layers, -(-512 * 2**20 // cache_bytes), (120 << 30) // cache_bytes))
+            m = HybridAttention(cfg, B, cap, "cuda", layers=n_cache)
+            for c in m.caches:
+                c.k.normal_(generator=gen)
+                c.v.normal_(generator=gen)
+            q = torch.randn(B, 32, 128, device="cuda", generator=gen).to(torch.bfloat16)
+            kn = torch.randn(B, 1, 8, 128, device="cuda", generator=gen).to(torch.bfloat16)
+            o = torch.empty_like(q)
+
+            def step():
+                for layer in range(n_layers):
+                    m.decode_layer(layer, q, kn, kn, o, cache_index=layer % n_cache)
+            for c in m.caches:
+                c.seq_len.fill_(T)
+            step()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            row = {"context": T, "batch": B, "distinct_caches": n_cache}
+            for f in fracs:
+                mask_for(m, B, f)
+                for c in m.caches:
+                    c.seq_len.fill_(T)
+                ms = graph_ms(graph, warm, reps)
+                row[f"{int(f * 100)}%"] = {"ms_per_step": ms, "tokens_per_s": B / (ms / 1e3)}
+            base = row["0%"]["ms_per_step"]
+            for f in fracs:
+                row[f"{int(f * 100)}%"]["speedup_vs_all_fa"] = base / row[f"{int(f * 100)}%"]["ms_per_step"]
+            row["fa_layer_ms"] = base / n_layers
+            row["sa_layer_ms"] = row["100%"]["ms_per_step"] / n_layers
+            out["decode"].append(row)
+            del graph, m, q, kn, o
+            torch.cuda.empty_cache()
+        # prefill: batch 1, 32 layers on separate caches whose lengths are views of one
+        # tensor, so a single memset in the graph restarts every layer at length 0
+        m = HybridAttention(cfg, 1, T, "cuda")
+        lens = torch.zeros(n_layers, 1, dtype=torch.int32, device="cuda")
+        for i, c in enumerate(m.caches):
+            c.seq_len = lens[i]
+        qp = torch.randn(1, T, 32, 128, device="cuda", generator=gen).to(torch.bfloat16)
+        kp = torch.randn(1, T, 8, 128, device="cuda", generator=gen).to(torch.bfloat16)
+        op = torch.empty_like(qp)
+
+        def pstep():
+            lens.zero_()
+            for layer in range(n_layers):
+                m.prefill_layer(layer, qp, kp, kp, op)
+        pstep()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            pstep()
+        row = {"context": T}
+        pw, pr = (1, 3) if T >= 65536 else (3, 5)
+        for f in fracs:
+            mask_for(m, 1, f)
+            ms = graph_ms(graph, pw, pr)
+            row[f"{int(f * 100)}%"] = {"ms": ms, "tokens_per_s": T / (ms / 1e3)}
+        base = row["0%"]["ms"]
+        for f in fracs:
+            row[f"{int(f * 100)}%"]["speedup_vs_all_fa"] = base / row[f"{int(f * 100)}%"]["ms"]
+        row["fa_layer_ms"] = base / n_layers
+        row["sa_layer_ms"] = row["100%"]["ms"] / n_layers
+        row["fa_tflops"] = prefill_flops_per_layer(cfg, T, True) / (row["fa_layer_ms"] / 1e3) / 1e12
+        out["prefill"].append(row)
+        del graph, m, lens, qp, kp, op
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    from sparse_attention_layer_b200 import flux
+    if flux.flux_get_device_status():
+        raise RuntimeError("device status set during the sweep")
+    print(json.dumps({"sweep": out, "measured": "graph-replayed 32-layer steps",
+                      "clocks": clocks}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -659,7 +778,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["flux", "reference"], default="flux")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--sweep", action="store_true",
+                    help="routing-mix x context x batch sweep (graph-replayed 32-layer steps)")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.warmup + args.steps > 256 - 1:
