@@ -5,9 +5,12 @@
 // cache [0, seq_len), SA reads only the sink rows and the window rows.  Decode is
 // bound by HBM bandwidth, so the kernel is built around moving K/V bytes:
 //
-//  * the visible keys of each (sequence, KV head) are cut into at most 64 splits of
-//    >= 128 keys; a persistent grid (one CTA per SM) walks the (sequence, KV head,
-//    split) items round-robin, so SA layers launch no idle CTAs;
+//  * the visible keys of each (sequence, KV head) pair are cut into 128-key stages;
+//    all pairs' stages, laid end to end, are dealt to the persistent grid (one CTA
+//    per SM) as equal contiguous ranges, so every CTA streams the same number of
+//    stages (FA and SA pairs, ragged lengths alike) and closes a partial result only
+//    where its range crosses a pair boundary -- one to three times per CTA at large
+//    batch, instead of once per fixed-size split;
 //  * one producer lane streams each split's K and V rows -- contiguous in the
 //    [B][Hkv][cap][d] cache -- into a 3-stage ring of 128-key stages with 1-D bulk
 //    copies (cp.async.bulk, no cluster), completing on mbarriers; the group's query
@@ -38,7 +41,7 @@ static __device__ __align__(256) unsigned char g_decode_static_scratch[FLUX_DECO
 namespace flux {
 namespace {
 
-constexpr int kStageKeys = 128;
+constexpr int kStageKeys = kDecStageKeys;
 constexpr int kMaxStages = 3;
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
@@ -55,11 +58,11 @@ struct DecodeArgs {
   const int32_t* seq_len;
   int batch, capacity, hkv, block, sink, window;
   float scale_log2;  // log2(e) / sqrt(d)
-  int min_splits;    // splits per (sequence, KV head) that give every SM 2 items
   int ring_rows;     // 0: contiguous cache; > 0: SA ring cache of sink + ring_rows rows
   int rows;          // physical rows per (sequence, KV head)
   float* ws_acc;     // [B][Hkv][kDecMaxSplits][G][D]
   float2* ws_ml;     // [B][Hkv][kDecMaxSplits][G] = (max, sum)
+  int* ws_nsplit;    // [B][Hkv]: partial results written for the pair
   uint16_t* o;
   unsigned* status;
 };
@@ -69,12 +72,12 @@ struct DecodeArgs {
 // contiguous cache's merged case), then [start1, start1 + len1) and
 // [start2, start2 + len2) (the window; two pieces when it wraps around a ring cache).
 struct Plan {
-  int n_vis, n_split, chunk;
+  int n_vis, stages;
   int len0, start1, len1, start2;
 };
 
 __device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
-  Plan p{0, 0, 1, 0, 0, 0, 0};
+  Plan p{0, 0, 0, 0, 0, 0};
   const int T = a.seq_len[b];
   if (T <= 0 || T > a.capacity) return p;
   const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
@@ -102,40 +105,50 @@ __device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
     }
   }
   p.n_vis = (r.hi0 - r.lo0) + (r.hi1 - r.lo1);
-  // splits: enough items for every SM (min_splits), at most kDecMaxChunk keys each
-  // when the split budget allows, never fewer than kDecMinChunk keys.
-  const int by_min = (p.n_vis + kDecMinChunk - 1) / kDecMinChunk;
-  const int by_max = (p.n_vis + kDecMaxChunk - 1) / kDecMaxChunk;
-  int s = by_max > a.min_splits ? by_max : a.min_splits;
-  if (s > by_min) s = by_min;
-  if (s > kDecMaxSplits) s = kDecMaxSplits;
-  p.n_split = s;
-  p.chunk = (p.n_vis + p.n_split - 1) / p.n_split;
+  p.stages = (p.n_vis + kDecStageKeys - 1) / kDecStageKeys;
   return p;
 }
 
+// One CTA's piece of one pair: the pair's stages [k0, k1) (virtual keys [v0, v1)).
+// split numbers the CTAs that share the pair, n_split counts them.
 struct Item {
-  int b, kvh, split;
-  int v0, v1;  // this split's virtual keys
+  int b, kvh, split, n_split;
+  int v0, v1;
+  int seg_end;  // global stage index where this piece ends
   Plan p;
 };
 
-// Item idx of the flattened (sequence, KV head, split) list; prefix[b] counts the
-// items of sequences before b.
-__device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix, int idx) {
+// The stage ranges: the pairs' stages laid end to end (sequence-major, then KV head),
+// prefix[b] = stages of all pairs of sequences before b; CTA c owns global stages
+// [c * per, (c + 1) * per).  per is at least ceil(max pair stages / 62), so a pair
+// meets at most 63 <= kDecMaxSplits CTAs.
+__device__ __forceinline__ int stages_per_cta(int total, int max_pair_stages) {
+  const int even = (total + int(gridDim.x) - 1) / int(gridDim.x);
+  const int cap = (max_pair_stages + kDecMaxSplits - 3) / (kDecMaxSplits - 2);
+  return max(1, max(even, cap));
+}
+
+// The piece that starts at global stage s of a range ending at end.
+__device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix, int s, int end,
+                                        int per) {
   int lo = 0, hi = a.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (prefix[mid] <= idx) lo = mid; else hi = mid;
+    if (prefix[mid] <= s) lo = mid; else hi = mid;
   }
   Item it;
   it.b = lo;
   it.p = make_plan(a, lo);
-  const int r = idx - prefix[lo];
-  it.kvh = r / it.p.n_split;
-  it.split = r % it.p.n_split;
-  it.v0 = it.split * it.p.chunk;
-  it.v1 = min(it.p.n_vis, it.v0 + it.p.chunk);
+  const int ns = it.p.stages;
+  const int r = s - prefix[lo];
+  it.kvh = r / ns;
+  const int pair0 = prefix[lo] + it.kvh * ns;
+  const int pair1 = pair0 + ns;
+  it.seg_end = min(end, pair1);
+  it.split = s / per - pair0 / per;
+  it.n_split = (pair1 - 1) / per - pair0 / per + 1;
+  it.v0 = (s - pair0) * kDecStageKeys;
+  it.v1 = min(it.p.n_vis, (it.seg_end - pair0) * kDecStageKeys);
   return it;
 }
 
@@ -252,7 +265,8 @@ struct DecodeSmemLayout {
   static constexpr size_t off_m = off_acc + size_t(kConsumerWarps) * G * D * 4;
   static constexpr size_t off_l = off_m + kConsumerWarps * G * 4;
   static constexpr size_t off_bar = (off_l + kConsumerWarps * G * 4 + 15) / 16 * 16;
-  static constexpr size_t off_prefix = off_bar + 2 * kStages * 8;
+  static constexpr size_t off_wmax = off_bar + 2 * kStages * 8;  // int per warp
+  static constexpr size_t off_prefix = off_wmax + 16 * 4;
   static size_t bytes(int batch) { return off_prefix + size_t(batch + 1) * 4; }
 };
 
@@ -278,20 +292,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
   float* sL = reinterpret_cast<float*>(smem + L::off_l);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   int* prefix = reinterpret_cast<int*>(smem + L::off_prefix);
+  int* wmax = reinterpret_cast<int*>(smem + L::off_wmax);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kStages);
 
-  // per-sequence item counts, then an exclusive scan (warp 0)
+  // per-sequence stage counts, then an exclusive scan (warp 0) and the largest pair
+  int my_max = 0;
   for (int b = tid; b < a.batch; b += kThreads) {
     const Plan p = make_plan(a, b);
-    prefix[b + 1] = a.hkv * p.n_split;
+    prefix[b + 1] = a.hkv * p.stages;
+    my_max = max(my_max, p.stages);
     const int T = a.seq_len[b];
     if ((T < 0 || T > a.capacity) && blockIdx.x == 0) atomicOr(a.status, kStatusBadLength);
     if (a.ring_rows > 0 && T > 0 && blockIdx.x == 0 &&
         route_is_fa(a.fa_mask, a.mask_words, b, a.layer))
       atomicOr(a.status, kStatusRingRoute);
   }
+  my_max = __reduce_max_sync(0xffffffffu, my_max);
+  if (lane == 0) wmax[warp] = my_max;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -314,9 +333,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       running += __shfl_sync(0xffffffffu, v, 31);
     }
     if (lane == 0) prefix[0] = 0;
+    int m = 0;
+    for (int w = 0; w < kThreads / 32; ++w) m = max(m, wmax[w]);
+    if (lane == 0) wmax[15] = m;
   }
   __syncthreads();
   const int total = prefix[a.batch];
+  const int per = stages_per_cta(total, wmax[15]);
+  const int range0 = min(total, int(blockIdx.x) * per);
+  const int range1 = min(total, range0 + per);
   const size_t row_elems = D;
 
   if (warp == kConsumerWarps) {
@@ -325,8 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       const uint64_t pol = l2_policy_evict_first();
       int g = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-        const Item it = item_at(a, prefix, idx);
+      for (int sg = range0; sg < range1 && ok;) {
+        const Item it = item_at(a, prefix, sg, range1, per);
+        sg = it.seg_end;
         const size_t head_off = (size_t(it.b) * a.hkv + it.kvh) * a.rows * row_elems;
         const uint16_t* qsrc = a.q + (size_t(it.b) * a.hkv * G + size_t(it.kvh) * G) * D;
         const int ns = item_stages(it);
@@ -367,8 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
   const int group_lane0 = lane & 24;
   int g = 0;
   bool ok = true;
-  for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-    const Item it = item_at(a, prefix, idx);
+  for (int sg = range0; sg < range1 && ok;) {
+    const Item it = item_at(a, prefix, sg, range1, per);
+    sg = it.seg_end;
     uint64_t q2[G][4 * NCH];   // pre-scaled query pairs of this lane's 8*NCH dims
     uint64_t acc[G][4 * NCH];  // P.V pairs of this lane's dims
 #pragma unroll
@@ -520,6 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
     }
     named_barrier_sync(1, kConsumerWarps * 32);
     const size_t rec = (size_t(it.b) * a.hkv + it.kvh) * kDecMaxSplits + it.split;
+    if (tid == 0 && it.split == 0) a.ws_nsplit[size_t(it.b) * a.hkv + it.kvh] = it.n_split;
     for (int i = tid; i < G * D; i += kConsumerWarps * 32) {
       const int h = i / D, e = i % D;
       float M = -INFINITY;
@@ -547,32 +575,32 @@ template <int D, int G>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
   __shared__ float wgt[kDecMaxSplits][G];
   const int kvh = blockIdx.x, b = blockIdx.y;
-  const Plan p = make_plan(a, b);
+  const int n_split = make_plan(a, b).n_vis > 0 ? a.ws_nsplit[size_t(b) * a.hkv + kvh] : 0;
   const size_t rec0 = (size_t(b) * a.hkv + kvh) * kDecMaxSplits;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   if (warp < G) {
     // one warp per query head of the group: splits spread over the lanes
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    if (lane < p.n_split) {
+    if (lane < n_split) {
       const float2 ml = a.ws_ml[(rec0 + lane) * G + warp];
       m0 = ml.x; l0 = ml.y;
     }
-    if (lane + 32 < p.n_split) {
+    if (lane + 32 < n_split) {
       const float2 ml = a.ws_ml[(rec0 + lane + 32) * G + warp];
       m1 = ml.x; l1 = ml.y;
     }
     float M = fmaxf(m0, m1);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float f0 = (lane < p.n_split) ? ex2_mufu(m0 - M) : 0.f;
-    const float f1 = (lane + 32 < p.n_split) ? ex2_mufu(m1 - M) : 0.f;
+    const float f0 = (lane < n_split) ? ex2_mufu(m0 - M) : 0.f;
+    const float f1 = (lane + 32 < n_split) ? ex2_mufu(m1 - M) : 0.f;
     float lv = f0 * l0 + f1 * l1;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, off);
     const float inv = (lv > 0.f) ? 1.f / lv : 0.f;
-    if (lane < p.n_split) wgt[lane][warp] = f0 * inv;
-    if (lane + 32 < p.n_split) wgt[lane + 32][warp] = f1 * inv;
+    if (lane < n_split) wgt[lane][warp] = f0 * inv;
+    if (lane + 32 < n_split) wgt[lane + 32][warp] = f1 * inv;
   }
   __syncthreads();
   uint16_t* out = a.o + (size_t(b) * a.hkv * G + size_t(kvh) * G) * D;
@@ -581,13 +609,13 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a)
     const float* src = a.ws_acc + (rec0 * G + gi) * D + e;
     float av0 = 0.f, av1 = 0.f, av2 = 0.f, av3 = 0.f;
     int s = 0;
-    for (; s + 4 <= p.n_split; s += 4) {
+    for (; s + 4 <= n_split; s += 4) {
       av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
       av1 = fmaf(wgt[s + 1][gi], src[size_t(s + 1) * G * D], av1);
       av2 = fmaf(wgt[s + 2][gi], src[size_t(s + 2) * G * D], av2);
       av3 = fmaf(wgt[s + 3][gi], src[size_t(s + 3) * G * D], av3);
     }
-    for (; s < p.n_split; ++s) av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
+    for (; s < n_split; ++s) av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
     const __nv_bfloat16 hb = __float2bfloat16_rn((av0 + av1) + (av2 + av3));
     out[gi * D + e] = *reinterpret_cast<const uint16_t*>(&hb);
   }
@@ -610,8 +638,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
-  const int max_items = a.batch * a.hkv * kDecMaxSplits;
-  const int grid = min(max_items, device_sm_count());
+  const int grid = device_sm_count();
   decode_split_kernel<D, G><<<grid, kThreads, smem, stream>>>(a);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -647,7 +674,7 @@ size_t decode_workspace_bytes(const AttnGeom& g, int batch) {
   const int G = g.hq / g.hkv;
   const size_t recs = size_t(batch) * g.hkv * kDecMaxSplits * G;
   const size_t acc = (recs * g.head_dim * 4 + 255) / 256 * 256;
-  return acc + recs * 8;
+  return acc + recs * 8 + size_t(batch) * g.hkv * 4;
 }
 
 cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
@@ -672,14 +699,11 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
   a.sink = g.sink;
   a.window = g.window;
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(g.head_dim)));
-  {
-    const int pairs = batch * g.hkv;
-    a.min_splits = (2 * device_sm_count() + pairs - 1) / pairs;
-  }
   const size_t recs = size_t(batch) * g.hkv * kDecMaxSplits * G;
   a.ws_acc = static_cast<float*>(workspace);
-  a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) +
-                                      (recs * g.head_dim * 4 + 255) / 256 * 256);
+  const size_t acc_bytes = (recs * g.head_dim * 4 + 255) / 256 * 256;
+  a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + acc_bytes);
+  a.ws_nsplit = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + acc_bytes + recs * 8);
   a.o = o;
   a.status = status;
 #define FLUX_DECODE_CASE(DD, GG) \

@@ -14,8 +14,7 @@ struct AttnGeom {
 
 // ----- decode (split-KV + combine)
 constexpr int kDecMaxSplits = 64;   // splits per (sequence, KV head)
-constexpr int kDecMinChunk = 128;   // fewest keys per split
-constexpr int kDecMaxChunk = 1024;  // most keys per split while the split budget allows
+constexpr int kDecStageKeys = 128;  // keys per decode pipeline stage
 constexpr int kDecMaxBatch = 1024;
 
 size_t decode_workspace_bytes(const AttnGeom& g, int batch);

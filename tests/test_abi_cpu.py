@@ -60,11 +60,12 @@ def _cfg(**kw):
 
 
 def test_workspace_size_formula(L):
-    # per (sequence, KV head, split, query head of the group): d fp32 partials + (max, sum)
+    # per (sequence, KV head, split, query head of the group): d fp32 partials + (max, sum),
+    # then one split count per (sequence, KV head)
     c = _cfg()
     got = L.flux_decode_workspace_size(ctypes.byref(c), 16)
     recs = 16 * 8 * 64 * 4
-    assert got == (recs * 128 * 4 + 255) // 256 * 256 + recs * 8
+    assert got == (recs * 128 * 4 + 255) // 256 * 256 + recs * 8 + 16 * 8 * 4
     bad = _cfg(head_dim=96)
     assert L.flux_decode_workspace_size(ctypes.byref(bad), 16) == 0
     assert L.flux_decode_workspace_size(ctypes.byref(c), 0) == 0
