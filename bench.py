@@ -255,16 +255,18 @@ class DecodeBench:
         for c in self.model.caches:
             c.seq_len.fill_(self.ctx)
 
-    def step(self, fa_events=None):
-        """One decode token for every sequence through all layers.  With fa_events, the
-        flux_decode call of every FA layer is bracketed by CUDA events."""
+    def step(self, fa_events=None, sa_events=None):
+        """One decode token for every sequence through all layers.  With fa_events /
+        sa_events, the flux_decode call of every FA / SA layer is bracketed by CUDA
+        events."""
         from sparse_attention_layer_b200 import flux
         m = self.model
         for layer in range(self.w.n_layers):
             c = m.caches[layer]
             flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, self.k_new[layer],
                                 self.v_new[layer])
-            timed = fa_events is not None and self.fa[layer]
+            events = fa_events if self.fa[layer] else sa_events
+            timed = events is not None
             if timed:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
@@ -273,9 +275,10 @@ class DecodeBench:
                              self.o[layer], m.workspace)
             if timed:
                 e1.record()
-                fa_events.append((e0, e1))
+                events.append((e0, e1))
 
-    launches_per_step = property(lambda self: self.w.n_layers * 4)  # append 2 + decode 2
+    # kernels of this library per step: append copy + advance, decode split + combine
+    launches_per_step = property(lambda self: self.w.n_layers * 4)
 
 
 class PrefillBench:
@@ -433,13 +436,13 @@ def run_flux(args, world, rank, local):
     sampler = ClockSampler(local)
     barrier(world)
     sampler.start()
-    fa_events = []
+    fa_events, sa_events = [], []
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     barrier(world)
     start.record()
     for _ in range(args.steps):
-        db.step(fa_events=fa_events)
+        db.step(fa_events=fa_events, sa_events=sa_events)
     end.record()
     barrier(world)
     st = flux.flux_get_device_status()
@@ -461,6 +464,14 @@ def run_flux(args, world, rank, local):
                 "launch_ms": statistics.mean(fa_ms),
                 "algorithmic_bytes_per_launch": fa_bytes}
     sa_bytes = decode_bytes_per_layer(w, cfg, int(round(T_mean)), False)
+    sa_ms = elapsed_ms(sa_events) if sa_events else None
+    roofline_sa = None if not sa_ms else {
+        "bound": "hbm", "kernel": "flux_decode (split-KV + combine), SA layers",
+        "achieved": sa_bytes / (statistics.mean(sa_ms) / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+        "unit": "GB/s",
+        "frac": sa_bytes / (statistics.mean(sa_ms) / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "peak_kind": f"{peak_kind} hbm_gbs", "launch_ms": statistics.mean(sa_ms),
+        "algorithmic_bytes_per_launch": sa_bytes}
     step_bytes = sum(decode_bytes_per_layer(w, cfg, int(round(T_mean)), fa) for fa in db.fa)
 
     # ---------------- decode as one CUDA graph per step (the headline number)
@@ -581,6 +592,7 @@ def run_flux(args, world, rank, local):
         "what": "the 16 SA layers' caches moved to rings of sink 128 + 2048 rows per "
                 "(sequence, KV head) after prefill; the same graph-replayed decode step",
     }
+    launches_per_step = db.launches_per_step
     del ring_graph, db
     torch.cuda.empty_cache()
 
@@ -639,12 +651,12 @@ def run_flux(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": decode_config(w, cfg, sa_layers),
-        "roofline": roofline,
+        "roofline": roofline, "roofline_sa": roofline_sa,
         "decode_step": {"algorithmic_gb_per_step": step_bytes / 1e9,
                         "step_gb_per_s": step_bytes / (ms_step / 1e3) / 1e9,
                         "fa_layer_bytes": fa_bytes, "sa_layer_bytes": sa_bytes},
         "cpu_baseline": cpu, "e2e": e2e, "decode_eager": eager,
-        "gpu_launches": w.n_layers * 4 * args.steps, "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
         "prefill": prefill, "routing_mix": mix, "sa_kv_eviction": eviction,
     }
     if rank == 0:
