@@ -296,6 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kStages);
+  pdl_trigger();  // the combine kernel may be scheduled now; it waits for this grid
+  pdl_wait();     // seq_len, the caches and the workspace come from earlier kernels
 
   // per-sequence stage counts, then an exclusive scan (warp 0) and the largest pair
   int my_max = 0;
@@ -574,6 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
 template <int D, int G>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
   __shared__ float wgt[kDecMaxSplits][G];
+  pdl_trigger();
+  pdl_wait();  // the split kernel's partials
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int n_split = make_plan(a, b).n_vis > 0 ? a.ws_nsplit[size_t(b) * a.hkv + kvh] : 0;
   const size_t rec0 = (size_t(b) * a.hkv + kvh) * kDecMaxSplits;
@@ -638,12 +642,10 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
-  const int grid = device_sm_count();
-  decode_split_kernel<D, G><<<grid, kThreads, smem, stream>>>(a);
-  err = cudaGetLastError();
+  err = launch_pdl(decode_split_kernel<D, G>, dim3(device_sm_count()), dim3(kThreads), smem,
+                   stream, a);
   if (err != cudaSuccess) return err;
-  decode_combine_kernel<D, G><<<dim3(a.hkv, a.batch), 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(decode_combine_kernel<D, G>, dim3(a.hkv, a.batch), dim3(256), 0, stream, a);
 }
 
 constexpr int kMaxDevices = 64;

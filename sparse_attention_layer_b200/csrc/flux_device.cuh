@@ -247,4 +247,17 @@ __device__ __forceinline__ void named_barrier_sync(int id, int n_threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n_threads) : "memory");
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// A kernel launched with programmatic stream serialisation may start while the
+// kernel before it on the stream is still running.  pdl_wait() blocks until that
+// kernel has completed and its memory is visible (a no-op for a normal launch);
+// every such kernel calls it before touching global memory.  pdl_trigger() lets the
+// next kernel on the stream be launched early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace flux

@@ -12,6 +12,26 @@ struct AttnGeom {
   int n_layers, mask_words, hq, hkv, head_dim, block, sink, window;
 };
 
+// Launch with programmatic dependent launch allowed (the kernel must call pdl_wait()
+// before its first global memory access): its CTAs can be scheduled while the
+// previous kernel on the stream drains, hiding launch latency between the short
+// kernels of a decode step.
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
+}
+
 // ----- decode (split-KV + combine)
 constexpr int kDecMaxSplits = 64;   // splits per (sequence, KV head)
 constexpr int kDecStageKeys = 128;  // keys per decode pipeline stage

@@ -5,9 +5,13 @@
 // in one contiguous byte range -- the property the decode bulk copies and the prefill
 // TMA boxes rely on (the pages' "contiguous memory access" of layer-level routing).
 //
-// Two launches: the copy reads seq_len[b] as the write position; the second launch
-// advances seq_len[b], so no copy CTA can observe a half-updated length.  A sequence
-// that would pass the capacity is skipped and FLUX_DEVICE_CAPACITY is set.
+// Large appends (prefill) take two launches: the copy reads seq_len[b] as the write
+// position; the second launch advances seq_len[b], so no copy CTA can observe a
+// half-updated length.  Small appends (decode: a few rows per sequence) take one: a
+// single CTA per sequence copies its rows and then advances seq_len[b] itself after a
+// CTA barrier; it is launched with programmatic dependent launch, like the decode
+// kernels after it.  A sequence that would pass the capacity is skipped and
+// FLUX_DEVICE_CAPACITY is set.
 //
 // SA ring caches (decode-time KV eviction of layers routed to SA): sink rows stay in
 // place and position p >= sink lives in row sink + (p - sink) mod ring_rows, so with
@@ -48,6 +52,38 @@ __global__ void __launch_bounds__(256) kv_append_copy_kernel(
   }
 }
 
+// One CTA per sequence: copy the rows, then advance the length (read by every thread
+// before the barrier, written by one thread after it).
+__global__ void __launch_bounds__(256) kv_append_fused_kernel(
+    uint16_t* __restrict__ k_cache, uint16_t* __restrict__ v_cache, int32_t* seq_len,
+    int capacity, const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
+    int n_new, int hkv, int chunks_per_row, unsigned* status) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x;
+  const int start = seq_len[b];
+  const bool fits = start >= 0 && start + n_new <= capacity;
+  if (fits) {
+    const int per_seq = n_new * hkv * chunks_per_row;
+    const size_t row_elems = size_t(chunks_per_row) * 8;
+    const uint4* ks = reinterpret_cast<const uint4*>(k_new) + size_t(b) * per_seq;
+    const uint4* vs = reinterpret_cast<const uint4*>(v_new) + size_t(b) * per_seq;
+    for (int i = threadIdx.x; i < per_seq; i += blockDim.x) {
+      const int ch = i % chunks_per_row;
+      const int rest = i / chunks_per_row;
+      const int kvh = rest % hkv;
+      const int tok = rest / hkv;
+      const size_t dst = ((size_t(b) * hkv + kvh) * capacity + start + tok) * row_elems + ch * 8;
+      *reinterpret_cast<uint4*>(k_cache + dst) = __ldg(ks + i);
+      *reinterpret_cast<uint4*>(v_cache + dst) = __ldg(vs + i);
+    }
+  } else if (threadIdx.x == 0) {
+    atomicOr(status, kStatusCapacity);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && fits) seq_len[b] = start + n_new;
+}
+
 __global__ void kv_append_advance_kernel(int32_t* seq_len, int batch, int capacity, int n_new) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
@@ -86,6 +122,36 @@ __global__ void __launch_bounds__(256) kv_append_ring_kernel(
     *reinterpret_cast<uint4*>(k_ring + dst) = __ldg(ks + i);
     *reinterpret_cast<uint4*>(v_ring + dst) = __ldg(vs + i);
   }
+}
+
+// Ring append of a few rows: one CTA per sequence, then it advances the length.
+__global__ void __launch_bounds__(256) kv_append_ring_fused_kernel(
+    uint16_t* __restrict__ k_ring, uint16_t* __restrict__ v_ring, int32_t* seq_len, int sink,
+    int ring_rows, const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
+    int n_new, int hkv, int chunks_per_row) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x;
+  const int start = seq_len[b];
+  if (start >= 0) {
+    const int rows = sink + ring_rows;
+    const int per_seq = n_new * hkv * chunks_per_row;
+    const size_t row_elems = size_t(chunks_per_row) * 8;
+    const uint4* ks = reinterpret_cast<const uint4*>(k_new) + size_t(b) * per_seq;
+    const uint4* vs = reinterpret_cast<const uint4*>(v_new) + size_t(b) * per_seq;
+    for (int i = threadIdx.x; i < per_seq; i += blockDim.x) {
+      const int ch = i % chunks_per_row;
+      const int rest = i / chunks_per_row;
+      const int kvh = rest % hkv;
+      const int tok = rest / hkv;
+      const int slot = ring_slot(start + tok, sink, ring_rows);
+      const size_t dst = ((size_t(b) * hkv + kvh) * rows + slot) * row_elems + ch * 8;
+      *reinterpret_cast<uint4*>(k_ring + dst) = __ldg(ks + i);
+      *reinterpret_cast<uint4*>(v_ring + dst) = __ldg(vs + i);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && start >= 0) seq_len[b] = start + n_new;
 }
 
 __global__ void kv_advance_unbounded_kernel(int32_t* seq_len, int batch, int n_new) {
@@ -129,12 +195,18 @@ __global__ void __launch_bounds__(256) kv_compact_ring_kernel(
 
 }  // namespace
 
+// Per-sequence rows (16-byte chunks) up to which one CTA per sequence does the append.
+constexpr long long kFusedAppendChunks = 4096;
+
 cudaError_t launch_kv_append_ring(const AttnGeom& g, uint16_t* k_ring, uint16_t* v_ring,
                                   int32_t* seq_len, int batch, int ring_rows,
                                   const uint16_t* k_new, const uint16_t* v_new, int n_new,
                                   cudaStream_t stream) {
   const int chunks = g.head_dim / 8;
   const long long per_seq = (long long)n_new * g.hkv * chunks;
+  if (per_seq <= kFusedAppendChunks)
+    return launch_pdl(kv_append_ring_fused_kernel, dim3(batch), dim3(256), 0, stream, k_ring,
+                      v_ring, seq_len, g.sink, ring_rows, k_new, v_new, n_new, g.hkv, chunks);
   long long blocks = (per_seq + 255) / 256;
   const long long cap_blocks = (long long)device_sm_count() * 16 / (batch > 0 ? batch : 1) + 1;
   if (blocks > cap_blocks) blocks = cap_blocks;
@@ -169,6 +241,9 @@ cudaError_t launch_kv_append(const AttnGeom& g, uint16_t* k_cache, uint16_t* v_c
                              cudaStream_t stream) {
   const int chunks = g.head_dim / 8;
   const long long per_seq = (long long)n_new * g.hkv * chunks;
+  if (per_seq <= kFusedAppendChunks)
+    return launch_pdl(kv_append_fused_kernel, dim3(batch), dim3(256), 0, stream, k_cache,
+                      v_cache, seq_len, capacity, k_new, v_new, n_new, g.hkv, chunks, status);
   long long blocks = (per_seq + 255) / 256;
   const long long cap_blocks = (long long)device_sm_count() * 16 / (batch > 0 ? batch : 1) + 1;
   if (blocks > cap_blocks) blocks = cap_blocks;
