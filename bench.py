@@ -277,8 +277,8 @@ class DecodeBench:
                 e1.record()
                 events.append((e0, e1))
 
-    # kernels of this library per step: append copy + advance, decode split + combine
-    launches_per_step = property(lambda self: self.w.n_layers * 4)
+    # kernels of this library per step: one-kernel append, decode split + combine
+    launches_per_step = property(lambda self: self.w.n_layers * 3)
 
 
 class PrefillBench:
@@ -493,7 +493,7 @@ def run_flux(args, world, rank, local):
     clocks = sampler.stop()  # sampled over the eager and the graph timed regions
     tg_ms = max_over_ranks(gs.elapsed_time(ge), world)
     eager = {"value": value, "ms_per_step": ms_step,
-             "what": "the same steps as 4 x 32 separate launches from Python"}
+             "what": "the same steps as 3 x 32 separate launches from Python"}
     value = replica_tokens_per_s(world, w.batch, args.steps, tg_ms)
     ms_step = tg_ms / args.steps
     st = flux.flux_get_device_status()
