@@ -116,6 +116,20 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Non-blocking test of an mbarrier phase (try_wait may suspend the thread for a while;
+// the MMA issuer polls two warpgroups and must not sleep on one of them).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -327,7 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
   const TilePlan plan = plan_tiles(a, fa, q_start + row0, q_start + row0 + rows - 1);
 
-  if (tid == 0) {
+  // The K producer thread initialises the barriers and issues the Q tile and the first
+  // K tiles at once, while the MMA warp allocates tensor memory: the loads are in
+  // flight before the CTA-wide barrier instead of after it.
+  const bool k_thread = (tid == kKProducerWarp * 32);
+  const int kv_row = b * a.hkv + kvh;
+  int k_pre = 0;  // K tiles issued before the barrier
+  if (k_thread) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar_kfull + 8 * s, 1);
@@ -345,6 +365,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_ofinal, 1);
     mbar_init(bar_idle, 1);
     fence_barrier_init();
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    mbar_arrive_expect_tx(bar_q, L::tile);
+    for (int c = 0; c < NCH; ++c) tma_load_4d(sQ + c * kSubBytes, &tmQ, c * 64, h, row0, b, bar_q);
+    k_pre = plan.n_tiles < kKStages ? plan.n_tiles : kKStages;
+    for (int j = 0; j < k_pre; ++j) {
+      const int k0 = tile_key0(plan, j);
+      mbar_arrive_expect_tx(bar_kfull + 8 * j, L::tile);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_3d(sK + j * L::tile + c * kSubBytes, &tmK, c * 64, k0, kv_row, bar_kfull + 8 * j);
+    }
   }
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -369,16 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t empty = is_k ? bar_kempty : bar_vempty;
       const uint32_t ring = is_k ? sK : sV;
       const CUtensorMap* map = is_k ? &tmK : &tmV;
-      prefetch_tmap(map);
-      if (is_k) {
-        prefetch_tmap(&tmQ);
-        mbar_arrive_expect_tx(bar_q, L::tile);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_4d(sQ + c * kSubBytes, &tmQ, c * 64, h, row0, b, bar_q);
-      }
-      const int kv_row = b * a.hkv + kvh;
-      int issued = 0;
-      for (int j = 0; j < plan.n_tiles; ++j) {
+      if (!is_k) prefetch_tmap(map);
+      // Q and the first K tiles were issued before the CTA barrier
+      int issued = is_k ? k_pre : 0;
+      for (int j = issued; j < plan.n_tiles; ++j) {
         const int st = j % n_st;
         const uint32_t ph = (j / n_st) & 1;
         if (!mbar_wait(empty + 8 * st, ph ^ 1, a.status)) break;
@@ -399,10 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = make_idesc(BM, BN, false, false);
       constexpr uint32_t idesc_o = make_idesc(BM, D, false, true);
       bool ok = mbar_wait(bar_q, 0, a.status);
-      // S_j = Q K_j^T into the S buffer of warpgroup j % 2
-      auto issue_s = [&](int j) -> bool {
+      // S_j = Q K_j^T into the S buffer of warpgroup j % 2 (its K stage has landed)
+      auto issue_s_ready = [&](int j) {
         const int st = j % kKStages;
-        if (!mbar_wait(bar_kfull + 8 * st, (j / kKStages) & 1, a.status)) return false;
         tc_fence_after();
         const uint32_t kb = sK + st * L::tile;
         const uint32_t sbuf = tmem + (j & 1) * 128;
@@ -414,27 +438,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar_sfull + 8 * (j & 1));
         mma_commit(bar_kempty + 8 * st);
-        return true;
       };
-      if (ok && plan.n_tiles > 0) ok = issue_s(0);
-      if (ok && plan.n_tiles > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < plan.n_tiles; ++j) {
-        const int g = j & 1;
-        const int st = j % kVStages;
-        if (!mbar_wait(bar_vfull + 8 * st, (j / kVStages) & 1, a.status)) break;
-        if (!mbar_wait(bar_pfull + 8 * g, (j >> 1) & 1, a.status)) break;
-        tc_fence_after();
-        const uint32_t vb = sV + st * L::tile;
-        const uint32_t pcol = tmem + g * 128;
+      auto k_ready = [&](int j) { return mbar_test(bar_kfull + 8 * (j % kKStages), (j / kKStages) & 1); };
+      const int n = plan.n_tiles;
+      for (int j = 0; ok && j < 2 && j < n; ++j) {
+        ok = mbar_wait(bar_kfull + 8 * (j % kKStages), (j / kKStages) & 1, a.status);
+        if (ok) issue_s_ready(j);
+      }
+      // Each warpgroup's P.V is issued as soon as its P (and V tile) is ready, in
+      // whichever order the two warpgroups finish: their O accumulators and S buffers
+      // are separate, and per warpgroup the order stays P_j V_j, S_{j+2}, P_{j+2} V_{j+2}.
+      // S_{j+2} overwrites P_j; MMAs issued by this thread execute in issue order, so
+      // P_j V_j has read its operand first.  Polling uses the non-blocking test.
+      int nxt[2] = {0, 1};       // next tile of each warpgroup waiting for its P.V
+      int pend[2] = {-1, -1};    // an S tile issued after the next K stage lands
+      unsigned long long t_last = global_ns();
+      while (ok && (nxt[0] < n || nxt[1] < n || pend[0] >= 0 || pend[1] >= 0)) {
+        bool progress = false;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_tmem_a(tmem + kTmemO + g * 128, pcol + kk * 8,
-                          sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o,
-                          (j >= 2 || kk > 0));
-        mma_commit(bar_vempty + 8 * st);
-        // S_{j+2} overwrites P_j.  MMAs issued by this thread execute in issue order,
-        // so P_j V_j has read its operand before S_{j+2} writes the buffer.
-        if (j + 2 < plan.n_tiles && !issue_s(j + 2)) break;
+        for (int g = 0; g < 2; ++g) {
+          if (pend[g] >= 0) {
+            if (!k_ready(pend[g])) continue;
+            issue_s_ready(pend[g]);
+            pend[g] = -1;
+            progress = true;
+          }
+          const int j = nxt[g];
+          if (j >= n) continue;
+          const int st = j % kVStages;
+          if (!mbar_test(bar_pfull + 8 * g, (j >> 1) & 1)) continue;
+          if (!mbar_test(bar_vfull + 8 * st, (j / kVStages) & 1)) continue;
+          tc_fence_after();
+          const uint32_t vb = sV + st * L::tile;
+          const uint32_t pcol = tmem + g * 128;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_bf16_tmem_a(tmem + kTmemO + g * 128, pcol + kk * 8,
+                            sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o,
+                            (j >= 2 || kk > 0));
+          mma_commit(bar_vempty + 8 * st);
+          nxt[g] = j + 2;
+          if (j + 2 < n) {
+            if (k_ready(j + 2)) issue_s_ready(j + 2);
+            else pend[g] = j + 2;
+          }
+          progress = true;
+        }
+        if (progress) {
+          t_last = global_ns();
+        } else if (global_ns() - t_last > kWaitLimitNs) {
+          atomicOr(a.status, kStatusTimeout);
+          ok = false;
+        }
       }
       // every MMA this thread issued has finished before tensor memory is freed
       mma_commit(bar_ofinal);
@@ -460,6 +515,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int k0 = tile_key0(plan, j);
       const bool masked = tile_needs_mask(plan, k0, a.sink);
+      // This row's visible key offsets i in [0, BN) of the tile: causal i <= lim, and for
+      // SA outside the gap [gap0, gap1) between the sink and the window (has_gap: the
+      // gap meets this tile).  The mask costs instructions on every key of a masked tile
+      // (the diagonal tile of every causal row block), so the common causal-only case is
+      // one compare and one select per key.
+      const int lim = t - k0;
+      const int gap0 = plan.fa ? BN : min(max(a.sink - k0, 0), BN);
+      const int gap1 = plan.fa ? BN : min(max(wl - k0, 0), BN);
+      const bool has_gap = __any_sync(0xffffffffu, gap0 < gap1);
       // Load 64 columns of the S row into s[] and apply the tile's mask.
       auto load_half = [&](uint32_t (&s)[64], int half) {
         FLUX_TMEM_LD32(srow + half * 64, s);
@@ -469,11 +533,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_ld();
         if (masked) {
+          const int lim_h = lim - half * 64;  // visible iff i <= lim_h
+          if (has_gap) {
+            const int g0 = gap0 - half * 64, g1 = gap1 - half * 64;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int jk = k0 + half * 64 + i;
-            const bool vis = (jk <= t) && (plan.fa || jk < a.sink || jk >= wl);
-            if (!vis) s[i] = __float_as_uint(-INFINITY);
+            for (int i = 0; i < 64; ++i) {
+              const bool vis = (i <= lim_h) & ((i < g0) | (i >= g1));
+              s[i] = vis ? s[i] : 0xff800000u;  // -inf
+            }
+          } else if (__any_sync(0xffffffffu, lim_h < 63)) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) s[i] = (i <= lim_h) ? s[i] : 0xff800000u;
           }
         }
       };
