@@ -64,6 +64,8 @@ typedef enum flux_status {
 #define FLUX_DEVICE_TIMEOUT 0x2u  /* a pipeline wait ran out of time; output invalid */
 #define FLUX_DEVICE_BAD_LENGTH 0x4u /* seq_len < n_q in prefill, or seq_len > capacity */
 #define FLUX_DEVICE_RING_ROUTE 0x8u /* flux_decode_ring saw a sequence routed to FA */
+#define FLUX_DEVICE_LAYOUT 0x10u    /* prefill: dynamic shared memory not 1024-byte aligned;
+                                       nothing computed (never seen on B200) */
 
 /* Attention geometry of one model; the same struct serves every layer. */
 typedef struct flux_attn_cfg {

@@ -19,6 +19,7 @@ constexpr unsigned kStatusCapacity = 0x1u;
 constexpr unsigned kStatusTimeout = 0x2u;
 constexpr unsigned kStatusBadLength = 0x4u;
 constexpr unsigned kStatusRingRoute = 0x8u;
+constexpr unsigned kStatusLayout = 0x10u;
 
 // A pipeline wait gives up after this long (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

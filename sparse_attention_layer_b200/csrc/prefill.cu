@@ -11,24 +11,28 @@
 //              memory (tcgen05.ld), masks boundary tiles, runs the online softmax in
 //              registers (log2 domain; its own stale row maximum, raised only when
 //              the new maximum exceeds it by more than 2^8, and then its O is
-//              rescaled in tensor memory) and writes P as bf16 back into tensor
-//              memory over its S columns, where the P.V MMA reads it as the A
-//              operand.  The exponentials are taken against the current maximum in
-//              the same pass that finds the tile maximum; only a warp with a row
-//              whose maximum jumped re-reads the tile.  Each warpgroup accumulates its own O; at the end the two
-//              partial (max, sum, O) are merged per row, normalised and stored.
+//              rescaled in tensor memory) and writes P as bf16 into its own P buffer
+//              in shared memory (128-byte swizzle, K-major: the A operand of P.V).
+//              As soon as the row of S has been read it releases the S buffer, so
+//              S_{j+2} runs on the tensor cores while the exponentials of tile j are
+//              still being computed.  The exponentials are taken against the current
+//              maximum in the same pass that finds the tile maximum; only a warp with a
+//              row whose maximum jumped re-reads the tile.  Each warpgroup accumulates
+//              its own O; at the end the two partial (max, sum, O) are merged per row,
+//              normalised and stored.
 //   warps 8-9  TMA producers (cp.async.bulk.tensor, 128-byte swizzle, no cluster, no
-//              multicast): warp 8 the Q tile once and K tiles into a 3-stage ring that
-//              is released as soon as each tile's S MMAs complete; warp 9 V tiles into
-//              a 2-stage ring released by the P.V MMAs.
-//   warp 10    MMA issuer (one thread): S_j = Q K_j^T (A, B from shared memory) into
-//              the S buffer of warpgroup j % 2, O_{j%2} += P_j V_j with P_j read from
-//              tensor memory and V_j an MN-major shared-memory operand; completion is
-//              signalled with tcgen05.commit on mbarriers.  S_{j+2} is issued right
-//              after P_j V_j: this thread's MMAs execute in issue order, so P_j has
-//              been read before S_{j+2} overwrites it.  The warp also allocates and
+//              multicast): warp 8 the Q tile once and K tiles into a ring (2 stages at
+//              d = 128, 3 at d = 64) released as soon as each tile's S MMAs complete;
+//              warp 9 V tiles into a 2-stage ring released by the P.V MMAs.
+//   warp 10    MMA issuer (one thread) with two streams per warpgroup: S_j = Q K_j^T
+//              (A, B from shared memory) into the S buffer of warpgroup j % 2 once that
+//              buffer is released and K_j has landed, and O_{j%2} += P_j V_j (P_j from
+//              the warpgroup's P buffer, V_j an MN-major operand) once P_j is written;
+//              completion is signalled with tcgen05.commit on mbarriers, the P buffer
+//              is released by the commit after P_j V_j.  The warp also allocates and
 //              frees the 512 tensor-memory columns (S0 | S1 | O0 | O1).
-// While one warpgroup runs its exponentials the tensor cores serve the other one.
+// Keeping P in tensor memory over S (the earlier design) forced S_{j+2} to wait for
+// P_j V_j; with P in shared memory the 8K-token FA launch went from 0.574 to 0.550 ms.
 //
 // Every mbarrier wait is bounded: on time-out the thread records FLUX_DEVICE_TIMEOUT
 // and leaves its loop; all roles meet at the final barrier, the producers first wait
@@ -45,8 +49,11 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (MMA M)
 constexpr int BN = 128;  // keys per KV tile (MMA N of Q K^T, MMA K of P V)
-constexpr int kKStages = 3;  // K tiles: released as soon as their S MMA completes
-constexpr int kVStages = 2;  // V tiles: released when their P.V MMA completes
+// K tiles are released as soon as their S MMA completes, V tiles when their P.V MMA
+// completes.  With P in shared memory (two 32 KB buffers) d = 128 fits 2 + 2 stages in
+// the 227 KB of a CTA; d = 64 keeps 3 K stages.
+template <int D> constexpr int kKSt = D == 128 ? 2 : 3;
+constexpr int kVStages = 2;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kKProducerWarp = 8;
 constexpr int kVProducerWarp = 9;
@@ -55,6 +62,7 @@ constexpr int kThreads = 352;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;           // O_g accumulator columns [256 + 128 g, + D)
 constexpr uint32_t kSubBytes = 128 * 128;  // one 64-column swizzled sub-tile of 128 rows
+constexpr uint32_t kPBytes = 2 * kSubBytes;  // P tile: 128 rows x 128 keys bf16
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 8 exponential pairs of a softmax row, this many go to the MUFU unit and the
 // rest to the polynomial on the FMA pipe.  Measured on B200 (Llama shape, 32K prompt):
@@ -67,19 +75,23 @@ struct Smem {
   static constexpr int NCH = D / 64;
   static constexpr uint32_t tile = NCH * kSubBytes;  // Q tile or one K / V tile
   static constexpr uint32_t off_q = 0;
+  static constexpr int KS = kKSt<D>;
   static constexpr uint32_t off_k = off_q + tile;
-  static constexpr uint32_t off_v = off_k + kKStages * tile;
-  static constexpr uint32_t off_ms = off_v + kVStages * tile;  // float [2][128] row maxima
+  static constexpr uint32_t off_v = off_k + KS * tile;
+  static constexpr uint32_t off_p = off_v + kVStages * tile;  // P of warpgroup g at + g kPBytes
+  static constexpr uint32_t off_ms = off_p + 2 * kPBytes;     // float [2][128] row maxima
   static constexpr uint32_t off_ls = off_ms + 2 * 128 * 4;      // float [2][128] row sums
   static constexpr uint32_t off_bar = off_ls + 2 * 128 * 4;
-  // q_full | k_full[3] | k_empty[3] | v_full[2] | v_empty[2] | s_full[2] | p_full[2] |
-  // o_done[2] | o_final | mma_idle
-  static constexpr int n_bars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2;
+  // q_full | k_full[KS] | k_empty[KS] | v_full[2] | v_empty[2] | s_full[2] | p_full[2] |
+  // s_free[2] | p_free[2] | o_final | mma_idle
+  static constexpr int n_bars = 1 + 2 * KS + 2 * kVStages + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t off_tmem = off_bar + n_bars * 8;
   static constexpr uint32_t used = off_tmem + 16;
-  // 1 KB slack to align the base; at least 116 KB so that a second CTA (which would
-  // need its own 512 tensor-memory columns) never shares the SM.
-  static constexpr uint32_t bytes = (used + 1024) > 118784 ? (used + 1024) : 118784;
+  // The dynamic shared memory starts 1024-byte aligned (checked by the kernel, which
+  // reports FLUX_DEVICE_LAYOUT otherwise), so no alignment slack is reserved: the d = 128
+  // layout needs 226 KB of the 227 KB a CTA may have.  At least 116 KB, so that a second
+  // CTA (which would need its own 512 tensor-memory columns) never shares the SM.
+  static constexpr uint32_t bytes = used > 118784 ? used : 118784;
 };
 
 struct PrefillArgs {
@@ -168,19 +180,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-
-// Same with the A operand (M x 16 bf16, one row per lane, pairs packed per column)
-// read from tensor memory.
-__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
@@ -300,11 +299,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
   using L = Smem<D>;
   constexpr int NCH = L::NCH;
+  constexpr int KS = L::KS;
   constexpr int DH = D / 2;  // O columns per softmax warpgroup
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (base - raw_addr);
+  if (raw_addr & 1023u) {  // the swizzled TMA tiles need 1024-byte alignment
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+      atomicOr(a.status, kStatusLayout);
+    return;
+  }
+  const uint32_t base = raw_addr;
+  uint8_t* smem = smem_raw;
 
   const uint32_t sQ = base + L::off_q;
   const uint32_t sK = base + L::off_k;
@@ -314,13 +319,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar0 = base + L::off_bar;
   const uint32_t bar_q = bar0;
   const uint32_t bar_kfull = bar0 + 8;                        // + 8 * K stage
-  const uint32_t bar_kempty = bar_kfull + 8 * kKStages;
-  const uint32_t bar_vfull = bar_kempty + 8 * kKStages;       // + 8 * V stage
+  const uint32_t bar_kempty = bar_kfull + 8 * KS;
+  const uint32_t bar_vfull = bar_kempty + 8 * KS;       // + 8 * V stage
   const uint32_t bar_vempty = bar_vfull + 8 * kVStages;
   const uint32_t bar_sfull = bar_vempty + 8 * kVStages;       // + 8 * warpgroup
   const uint32_t bar_pfull = bar_sfull + 16;                  // + 8 * warpgroup
-  const uint32_t bar_odone = bar_pfull + 16;                  // + 8 * warpgroup
-  const uint32_t bar_ofinal = bar_odone + 16;
+  const uint32_t bar_sfree = bar_pfull + 16;   // + 8 * warpgroup: S read, buffer reusable
+  const uint32_t bar_pfree = bar_sfree + 16;   // + 8 * warpgroup: P.V done, P buffer free
+  const uint32_t bar_ofinal = bar_pfree + 16;
+  const uint32_t sP = base + L::off_p;
   const uint32_t bar_idle = bar_ofinal + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_tmem);
 
@@ -349,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int k_pre = 0;  // K tiles issued before the barrier
   if (k_thread) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(bar_kfull + 8 * s, 1);
       mbar_init(bar_kempty + 8 * s, 1);
     }
@@ -360,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar_sfull + 8 * g, 1);
       mbar_init(bar_pfull + 8 * g, 4);
-      mbar_init(bar_odone + 8 * g, 1);
+      mbar_init(bar_sfree + 8 * g, 4);
+      mbar_init(bar_pfree + 8 * g, 1);
     }
     mbar_init(bar_ofinal, 1);
     mbar_init(bar_idle, 1);
@@ -369,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmK);
     mbar_arrive_expect_tx(bar_q, L::tile);
     for (int c = 0; c < NCH; ++c) tma_load_4d(sQ + c * kSubBytes, &tmQ, c * 64, h, row0, b, bar_q);
-    k_pre = plan.n_tiles < kKStages ? plan.n_tiles : kKStages;
+    k_pre = plan.n_tiles < KS ? plan.n_tiles : KS;
     for (int j = 0; j < k_pre; ++j) {
       const int k0 = tile_key0(plan, j);
       mbar_arrive_expect_tx(bar_kfull + 8 * j, L::tile);
@@ -395,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ring's release barriers, so K runs up to three tiles ahead of the MMAs.
     if (lane == 0) {
       const bool is_k = (warp == kKProducerWarp);
-      const int n_st = is_k ? kKStages : kVStages;
+      const int n_st = is_k ? KS : kVStages;
       const uint32_t full = is_k ? bar_kfull : bar_vfull;
       const uint32_t empty = is_k ? bar_kempty : bar_vempty;
       const uint32_t ring = is_k ? sK : sV;
@@ -425,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = make_idesc(BM, D, false, true);
       bool ok = mbar_wait(bar_q, 0, a.status);
       // S_j = Q K_j^T into the S buffer of warpgroup j % 2 (its K stage has landed)
-      auto issue_s_ready = [&](int j) {
-        const int st = j % kKStages;
+      auto issue_s = [&](int j) {
+        const int st = j % KS;
         tc_fence_after();
         const uint32_t kb = sK + st * L::tile;
         const uint32_t sbuf = tmem + (j & 1) * 128;
@@ -439,49 +447,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_sfull + 8 * (j & 1));
         mma_commit(bar_kempty + 8 * st);
       };
-      auto k_ready = [&](int j) { return mbar_test(bar_kfull + 8 * (j % kKStages), (j / kKStages) & 1); };
       const int n = plan.n_tiles;
       for (int j = 0; ok && j < 2 && j < n; ++j) {
-        ok = mbar_wait(bar_kfull + 8 * (j % kKStages), (j / kKStages) & 1, a.status);
-        if (ok) issue_s_ready(j);
+        ok = mbar_wait(bar_kfull + 8 * (j % KS), (j / KS) & 1, a.status);
+        if (ok) issue_s(j);
       }
-      // Each warpgroup's P.V is issued as soon as its P (and V tile) is ready, in
-      // whichever order the two warpgroups finish: their O accumulators and S buffers
-      // are separate, and per warpgroup the order stays P_j V_j, S_{j+2}, P_{j+2} V_{j+2}.
-      // S_{j+2} overwrites P_j; MMAs issued by this thread execute in issue order, so
-      // P_j V_j has read its operand first.  Polling uses the non-blocking test.
-      int nxt[2] = {0, 1};       // next tile of each warpgroup waiting for its P.V
-      int pend[2] = {-1, -1};    // an S tile issued after the next K stage lands
+      // Two independent streams per warpgroup g: S_{j+2} as soon as the softmax has read
+      // S_j out of tensor memory (s_free) and K_{j+2} has landed -- P lives in shared
+      // memory, so the S buffer is free before P_j V_j runs -- and P_j V_j as soon as P_j
+      // (p_full) and V_j have landed.  Polling uses the non-blocking test.
+      int s_next[2] = {2, 3}, pv_next[2] = {0, 1};
       unsigned long long t_last = global_ns();
-      while (ok && (nxt[0] < n || nxt[1] < n || pend[0] >= 0 || pend[1] >= 0)) {
+      while (ok && (pv_next[0] < n || pv_next[1] < n)) {
         bool progress = false;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          if (pend[g] >= 0) {
-            if (!k_ready(pend[g])) continue;
-            issue_s_ready(pend[g]);
-            pend[g] = -1;
+          const int js = s_next[g];
+          if (js < n && mbar_test(bar_sfree + 8 * g, ((js - 2) >> 1) & 1) &&
+              mbar_test(bar_kfull + 8 * (js % KS), (js / KS) & 1)) {
+            issue_s(js);
+            s_next[g] = js + 2;
             progress = true;
           }
-          const int j = nxt[g];
+          const int j = pv_next[g];
           if (j >= n) continue;
           const int st = j % kVStages;
           if (!mbar_test(bar_pfull + 8 * g, (j >> 1) & 1)) continue;
           if (!mbar_test(bar_vfull + 8 * st, (j / kVStages) & 1)) continue;
           tc_fence_after();
           const uint32_t vb = sV + st * L::tile;
-          const uint32_t pcol = tmem + g * 128;
+          const uint32_t pb = sP + g * kPBytes;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_tmem_a(tmem + kTmemO + g * 128, pcol + kk * 8,
-                            sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o,
-                            (j >= 2 || kk > 0));
-          mma_commit(bar_vempty + 8 * st);
-          nxt[g] = j + 2;
-          if (j + 2 < n) {
-            if (k_ready(j + 2)) issue_s_ready(j + 2);
-            else pend[g] = j + 2;
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+            mma_bf16(tmem + kTmemO + g * 128, sw128_desc(pb + off, 16, 1024),
+                     sw128_desc(vb + kk * 16 * 128, kSubBytes, 1024), idesc_o, (j >= 2 || kk > 0));
           }
+          mma_commit(bar_vempty + 8 * st);
+          mma_commit(bar_pfree + 8 * g);
+          pv_next[g] = j + 2;
           progress = true;
         }
         if (progress) {
@@ -506,6 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t srow = tmem + g * 128 + lane_base;
     const uint32_t orow = tmem + kTmemO + g * 128 + lane_base;
+    // this row of the warpgroup's P buffer (128-byte swizzle, K-major, as the MMA reads it)
+    const uint32_t prow = sP + g * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
     const float c = a.scale_log2;
     float m_used = -INFINITY;  // scaled (log2) units
     float l_sum = 0.f;
@@ -583,7 +589,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           f2_unpack(p2, p0, p1);
           pk[w] = pack_bf16x2(p0, p1);
         }
-        FLUX_TMEM_ST32(srow + half * 32, pk);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          sts128(prow + half * kSubBytes + ((cc ^ (r & 7)) << 4), pk[4 * cc], pk[4 * cc + 1],
+                 pk[4 * cc + 2], pk[4 * cc + 3]);
         const uint64_t sum2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         float s0, s1;
         f2_unpack(sum2, s0, s1);
@@ -592,6 +601,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Fast path: exponentials against the current stale maximum, one TMEM read of S.
       // Any row of the warp whose maximum moved by more than the threshold (and the
       // first tile) sends the warp to the slow path, which recomputes the tile.
+      // P_{j-2} V_{j-2} must have read this warpgroup's P buffer (and written O_g)
+      // before P_j is stored or O_g rescaled; waited for once, where first needed
+      bool p_free = false;
+      auto wait_p_free = [&]() {
+        if (!p_free) {
+          if (!mbar_wait(bar_pfree + 8 * g, ((j >> 1) & 1) ^ 1, a.status)) ok = false;
+          p_free = true;
+        }
+      };
+      // S_j has been read out of tensor memory: S_{j+2} may be issued into the buffer
+      auto release_s = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sfree + 8 * g);
+      };
       float mrow, lpart = 0.f;
       bool slow;
       {
@@ -600,12 +624,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mrow = max_half(s);
         slow = __any_sync(0xffffffffu, m_used == -INFINITY || mrow * c > m_used + kRescaleThreshold);
         if (!slow) {
+          wait_p_free();
           lpart = exp_half(s, 0, m_used);
           load_half(s, 1);
           const float m1 = max_half(s);
           mrow = fmaxf(mrow, m1);
           slow = __any_sync(0xffffffffu, m1 * c > m_used + kRescaleThreshold);
-          if (!slow) lpart += exp_half(s, 1, m_used);
+          if (!slow) {
+            release_s();
+            lpart += exp_half(s, 1, m_used);
+          }
         } else {
           load_half(s, 1);
           mrow = fmaxf(mrow, max_half(s));
@@ -621,8 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_tile;
           l_sum *= alpha;
         }
-        // O_g was last written by P_{j-2} V_{j-2}; the commit that signalled S_j
-        // covers it, so it has completed
+        // O_g was last written by P_{j-2} V_{j-2}: wait for it before the rescale
+        wait_p_free();
         if (j >= 2 && __any_sync(0xffffffffu, bump)) {
 #pragma unroll
           for (int q = 0; q < D / 32; ++q) {
@@ -640,11 +668,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int half = 0; half < 2; ++half) {
           uint32_t s[64];
           load_half(s, half);
+          if (half == 1) release_s();
           lpart += exp_half(s, half, m_use);
         }
       }
       l_sum += lpart;
       tmem_wait_st();
+      fence_proxy_async_smem();  // P stores, before the MMA reads them
       // keys past the valid length: zero their V rows (the cache there is unwritten)
       if (k0 + BN > seq) {
         const int st = j % kVStages;

@@ -29,6 +29,7 @@ FLUX_DEVICE_CAPACITY = 0x1
 FLUX_DEVICE_TIMEOUT = 0x2
 FLUX_DEVICE_BAD_LENGTH = 0x4
 FLUX_DEVICE_RING_ROUTE = 0x8
+FLUX_DEVICE_LAYOUT = 0x10
 
 # every entry point declared in include/flux.h
 EXPORTED = (
