@@ -625,10 +625,14 @@ def run_flux(args, world, rank, local):
         "ms_per_step": pf_step, "steps": n_pf, "sa_layers": pb.w.n_layers - n_fa,
         "router_ms": statistics.mean(elapsed_ms(rt_ev)),
         "algorithmic_tflops_per_step": (n_fa * flops_fa + (pb.w.n_layers - n_fa) * flops_sa) / 1e12,
+        # The FA launches are timed inside back-to-back 32-layer prefill steps (GPU busy
+        # for the whole phase, at the power cap), so the peak is the sustained one; the
+        # fraction of the burst peak (a kernel timed alone) is given beside it.
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128> (tcgen05), FA layers",
-                     "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": tflops / peaks["bf16_tflops"],
-                     "peak_kind": f"{peak_kind} bf16_tflops (burst)",
+                     "achieved": tflops, "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops_sustained"],
+                     "peak_kind": f"{peak_kind} bf16_tflops_sustained (timed inside a long step)",
+                     "frac_of_burst_peak": tflops / peaks["bf16_tflops"],
                      "traffic": measured_traffic("prefill", pb.w.batch),
                      "launch_ms": fa_launch, "algorithmic_flops_per_launch": flops_fa},
         "gpu_launches_per_step": pb.launches_per_step,
