@@ -31,6 +31,21 @@ def test_header_and_binding_agree():
     assert header_functions() == sorted(flux.EXPORTED)
 
 
+def test_status_constants_agree():
+    """Every device status bit and status code the header defines has the same value in
+    the binding (the tests and bench.py read them from there)."""
+    with open(os.path.join(ROOT, "include", "flux.h")) as f:
+        text = f.read()
+    bits = dict(re.findall(r"#define (FLUX_DEVICE_[A-Z_]+) (0x[0-9a-fA-F]+)u", text))
+    codes = dict(re.findall(r"\b(FLUX_(?:OK|ERR_[A-Z_]+)) = (\d+)", text))
+    assert len(bits) >= 5 and len(codes) >= 7
+    for name, val in bits.items():
+        assert getattr(flux, name) == int(val, 16), name
+    for name, val in codes.items():
+        assert getattr(flux, name) == int(val), name
+    assert len(set(int(v, 16) for v in bits.values())) == len(bits)  # distinct bits
+
+
 def test_library_exports_every_header_symbol(L):
     for name in header_functions():
         assert hasattr(L, name), f"libflux.so does not export {name}"
