@@ -369,6 +369,30 @@ def cpu_oracle_decode_sample(n_seq: int = 1, seed: int = 5):
     return out
 
 
+def cpu_oracle_prefill_sample(n_rows: int = 16, seed: int = 9):
+    """Time the fp64 oracle on n_rows query rows, evenly spaced over the Llama
+    8192-token prompt, of one FA and one SA layer (all 32 heads); returns seconds per
+    query row per layer for each route."""
+    import numpy as np
+
+    from oracle import flux_oracle as orc
+    from sparse_attention_layer_b200 import configs, inputs
+    w = configs.LLAMA_PREFILL
+    S = w.seq
+    q = inputs.normal_bf16((1, S, w.n_q_heads, w.head_dim), seed).float().numpy().astype(np.float64)
+    shape = (1, w.n_kv_heads, S, w.head_dim)
+    kc = inputs.normal_bf16(shape, seed + 1).float().numpy().astype(np.float64)
+    vc = inputs.normal_bf16(shape, seed + 2).float().numpy().astype(np.float64)
+    rows = np.linspace(0, S - 1, n_rows).astype(np.int64)
+    out = {}
+    for fa in (True, False):
+        t0 = time.perf_counter()
+        orc.attention_layer(q, kc, vc, np.array([S]), np.array([fa]), w.block, w.sink, w.window,
+                            rows=rows)
+        out[fa] = (time.perf_counter() - t0) / n_rows
+    return out
+
+
 def cpu_baseline_decode_tok_s(w, n_sa, n_seq=2):
     per = cpu_oracle_decode_sample(n_seq)
     per_seq_step = (w.n_layers - n_sa) * per[True] + n_sa * per[False]
@@ -636,7 +660,21 @@ def run_flux(args, world, rank, local):
                      "traffic": measured_traffic("prefill", pb.w.batch),
                      "launch_ms": fa_launch, "algorithmic_flops_per_launch": flops_fa},
         "gpu_launches_per_step": pb.launches_per_step,
+        "cpu_baseline": None,
     }
+    if world == 1 and rank == 0 and not args.no_cpu:
+        # the oracle on sampled query rows, extrapolated to the whole prompt (every row of
+        # 32 layers with this step's routes); a baseline, not a target
+        t0 = time.perf_counter()
+        per_row = cpu_oracle_prefill_sample()
+        sec = pb.w.seq * (n_fa * per_row[True] + (pb.w.n_layers - n_fa) * per_row[False])
+        prefill["cpu_baseline"] = {
+            "value": pb.w.seq / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "extrapolated": True,
+            "sample": "16 evenly spaced query rows x 32 heads of one FA and one SA layer of the "
+                      "8192-token prompt (fp64 oracle), extrapolated to all rows of "
+                      f"{n_fa} FA + {pb.w.n_layers - n_fa} SA layers; "
+                      f"{time.perf_counter() - t0:.1f} s of CPU time"}
     del pb
     torch.cuda.empty_cache()
 
