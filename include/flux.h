@@ -115,7 +115,11 @@ int flux_route(const flux_router_weights* w, const uint16_t* xq, int32_t batch,
  *                     [seq_len[b], seq_len[b] + n_new) and seq_len[b] += n_new.
  *   k_new, v_new      [batch][n_new][n_kv_heads][head_dim] bf16.
  * A sequence with seq_len[b] + n_new > capacity is left untouched (rows and
- * length) and FLUX_DEVICE_CAPACITY is set.  Two launches: copy, then length update.
+ * length) and FLUX_DEVICE_CAPACITY is set.  Up to 4096 16-byte chunks of new rows per
+ * sequence (decode-sized appends): one launch, a CTA per sequence that copies its rows
+ * and then advances its length (programmatic dependent launch, so it may start while
+ * the previous kernel on the stream drains); larger appends: a copy launch, then a
+ * length-update launch.
  */
 int flux_kv_append(const flux_attn_cfg* cfg, uint16_t* k_cache, uint16_t* v_cache,
                    int32_t* seq_len, int32_t batch, int32_t capacity,
@@ -131,9 +135,10 @@ int flux_kv_append(const flux_attn_cfg* cfg, uint16_t* k_cache, uint16_t* v_cach
  *            position t = seq_len[b] - n_q + i.
  *   k_cache, v_cache, seq_len  as written by flux_kv_append (seq_len read only).
  *   o        [batch][n_q][n_q_heads][head_dim] bf16, written.
- * tcgen05 / TMEM tensor-core kernel fed by TMA; SA visits only the sink and window
- * KV tiles.  seq_len[b] < n_q or > capacity sets FLUX_DEVICE_BAD_LENGTH and leaves
- * that sequence's output unwritten.
+ * tcgen05 / TMEM tensor-core kernel fed by TMA (two softmax warpgroups, P staged in
+ * shared memory; 226 KB of shared memory per CTA at head_dim 128); SA visits only the
+ * sink and window KV tiles.  seq_len[b] < n_q or > capacity sets
+ * FLUX_DEVICE_BAD_LENGTH and leaves that sequence's output unwritten.
  */
 int flux_prefill(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
                  const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
