@@ -109,7 +109,9 @@ int flux_route(const flux_router_weights* w, const uint16_t* xq, int32_t batch,
                double* logits, void* stream);
 
 /*
- * flux_kv_append -- append n_new rows per sequence to one layer's KV cache.
+ * flux_kv_append -- append n_new rows per sequence to one layer's KV cache: the
+ * persistent decode-time KV cache whose per-layer size Tables 15/16 report (the keys
+ * and values every later FA or SA query of that layer reads).
  *   k_cache, v_cache  [batch][n_kv_heads][capacity][head_dim] bf16 (read/write).
  *   seq_len           [batch] int32 (read/write): rows are written at positions
  *                     [seq_len[b], seq_len[b] + n_new) and seq_len[b] += n_new.
@@ -182,7 +184,10 @@ int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask
  *   FLUX_DECODE_STATIC_SCRATCH_BYTES returns FLUX_ERR_WORKSPACE without launching
  *   (the Llama-3.1-8B decode geometry fits up to batch 31).
  *   The first call on a device looks up the array's device address (with that
- *   device current) and caches it; make that first call before any stream capture.
+ *   device current) and caches it.  Under CUDA's lazy module loading (the default)
+ *   that first use is also when the device loads the library's decode module and so
+ *   reserves the array: make a first (warm-up) call at initialisation, while
+ *   allocation is still allowed, and before any stream capture.
  *   All calls share the one array, so calls that can overlap on the GPU (different
  *   streams, or devices sharing a context) race and corrupt each other's results;
  *   serialise them.  The array keeps the last call's contents; nothing in it needs to
@@ -237,6 +242,27 @@ int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa
  */
 int flux_sa_block_ranges(const flux_attn_cfg* cfg, int32_t n_qblocks, int32_t* ranges,
                          void* stream);
+
+/*
+ * flux_prefill_tile_plan -- the KV tiles flux_prefill visits, for checking the SA
+ * block indices of the prefill kernel exactly (streaming pattern of Table 6: sink
+ * blocks plus a local window of blocks, Figure 1 caption).  Same arguments as
+ * flux_prefill minus q, the caches and o; computed on the device by the tile schedule
+ * the prefill kernel itself runs.
+ *   tiles      [batch][ceil(n_q / 128)][max_tiles] int32 device memory, written: entry
+ *              i of query tile m (queries m*128 .. m*128 + 127 of the prompt) is the
+ *              index kt of the i-th 128-key tile (keys kt*128 .. kt*128 + 127) the
+ *              kernel visits for it, OR FLUX_TILE_MASKED when the kernel applies the
+ *              per-key mask in that tile (some query of the tile does not see some key
+ *              of it); -1 after the last visited tile.
+ *   max_tiles  >= ceil(capacity / 128), else FLUX_ERR_INVALID_ARG.
+ * A sequence with seq_len[b] < n_q or > capacity gets only -1 entries and sets
+ * FLUX_DEVICE_BAD_LENGTH, as flux_prefill would.
+ */
+#define FLUX_TILE_MASKED 0x40000000
+int flux_prefill_tile_plan(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                           const int32_t* seq_len, int32_t batch, int32_t capacity, int32_t n_q,
+                           int32_t* tiles, int32_t max_tiles, void* stream);
 
 /* flux_selftest_wait_timeout -- failure-detection self-test (the paper has no
  * counterpart): one thread waits on an mbarrier that nothing releases, through the

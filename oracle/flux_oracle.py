@@ -203,6 +203,21 @@ def sa_visible_key_blocks(qb: int, n_key_blocks: int, block: int, sink: int,
     return out
 
 
+def key_tiles_of_rows(is_fa: bool, q_pos: np.ndarray, tile: int, block: int, sink: int,
+                      window: int):
+    """Key tiles of `tile` keys that a block-sparse kernel must visit for the query rows
+    q_pos taken together, from the dense mask: the tiles holding a key visible from at
+    least one row, and, of those, the tiles where some (row, key) pair is not visible
+    (the kernel has to mask inside them).  Returns (visited, masked) as sorted lists."""
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    n_tiles = int(q_pos.max()) // tile + 1
+    mask = visible_mask(is_fa, q_pos, n_tiles * tile, block, sink, window)
+    per_tile = mask.reshape(len(q_pos), n_tiles, tile)
+    visited = [kt for kt in range(n_tiles) if per_tile[:, kt, :].any()]
+    masked = [kt for kt in visited if not per_tile[:, kt, :].all()]
+    return visited, masked
+
+
 # --------------------------------------------------------------------------------------
 # Attention (Table 6: FA dense path and SA streaming path; grouped-query KV sharing)
 # --------------------------------------------------------------------------------------

@@ -13,16 +13,15 @@
   seed chosen for 22 SA layers.
 * SWEEP: Llama shape over contexts x decode batches x SA-layer fractions.
 
-The router seeds for LLAMA_PREFILL and QWEN_PREFILL are recorded in
-tests/golden/router_seeds.json, written by tests/golden/make_router_seeds.py from the
-oracle alone.
+The router seeds of LLAMA_PREFILL (10) and QWEN_PREFILL (19) are the first seeds whose
+random-init router sends exactly 16 of 32 and 22 of 36 layers to SA at tau = 0 (the
+"~50%" and "~60%" SA workloads); a seed search over the fp64 oracle recorded them with
+the resulting bits, and the test suite checks these constants against that record.
 """
 
 from __future__ import annotations
 
 import dataclasses
-import json
-import os
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,14 +55,9 @@ class Workload:
         return self.seq + self.decode_steps
 
 
-def _router_seed(name: str, default: int) -> int:
-    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                        "tests", "golden", "router_seeds.json")
-    try:
-        with open(path) as f:
-            return int(json.load(f)[name]["router_seed"])
-    except (OSError, KeyError, ValueError):
-        return default
+# first router seeds giving exactly the target number of SA layers (see the module text)
+LLAMA_PREFILL_ROUTER_SEED = 10
+QWEN_PREFILL_ROUTER_SEED = 19
 
 
 TINY = Workload(
@@ -74,7 +68,7 @@ TINY = Workload(
 LLAMA_PREFILL = Workload(
     name="llama31_8b_prefill_8k", batch=1, n_layers=32, n_q_heads=32, n_kv_heads=8,
     head_dim=128, seq=8192, block=128, sink=128, window=2048, router_hidden=4096,
-    router_rank=256, data_seed=21, router_seed=_router_seed("llama31_8b_prefill_8k", 0),
+    router_rank=256, data_seed=21, router_seed=LLAMA_PREFILL_ROUTER_SEED,
     target_sa_layers=16)
 
 LLAMA_DECODE = Workload(
@@ -86,7 +80,7 @@ LLAMA_DECODE = Workload(
 QWEN_PREFILL = Workload(
     name="qwen3_4b_prefill_128k", batch=1, n_layers=36, n_q_heads=32, n_kv_heads=8,
     head_dim=128, seq=131072, block=128, sink=128, window=4096, router_hidden=2560,
-    router_rank=256, data_seed=41, router_seed=_router_seed("qwen3_4b_prefill_128k", 0),
+    router_rank=256, data_seed=41, router_seed=QWEN_PREFILL_ROUTER_SEED,
     target_sa_layers=22)
 
 # decode config's fixed mask: the first 16 entries of a seeded permutation of 32 layers

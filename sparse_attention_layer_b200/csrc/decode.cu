@@ -629,18 +629,24 @@ template <int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   using L = DecodeSmem<D, G>;
   const size_t smem = L::bytes(a.batch);
-  // the attribute is per device; set it (to the largest size any batch needs) once
+  // the attribute is per device; set it (to the largest size any batch needs) once.
+  // Host threads may make their first call on a device concurrently: the flag is
+  // read and written under a lock.
+  static std::mutex attr_mutex;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
-    err = cudaFuncSetAttribute(decode_split_kernel<D, G>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(L::bytes(kDecMaxBatch)));
-    if (err != cudaSuccess) return err;
-    attr_set[dev] = true;
+  {
+    std::lock_guard<std::mutex> lock(attr_mutex);
+    if (!attr_set[dev]) {
+      err = cudaFuncSetAttribute(decode_split_kernel<D, G>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(L::bytes(kDecMaxBatch)));
+      if (err != cudaSuccess) return err;
+      attr_set[dev] = true;
+    }
   }
   err = launch_pdl(decode_split_kernel<D, G>, dim3(device_sm_count()), dim3(kThreads), smem,
                    stream, a);

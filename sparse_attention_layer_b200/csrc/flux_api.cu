@@ -99,6 +99,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? FLUX_OK : FLUX_ERR_CU
 int device_sm_count() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(g_mutex);
   if (!g_sm_count[dev]) {
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
@@ -316,6 +317,25 @@ int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa
   return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_ring, v_ring, seq_len,
                                                batch, 0, ring_rows, o, workspace, status,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+int flux_prefill_tile_plan(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                           const int32_t* seq_len, int32_t batch, int32_t capacity, int32_t n_q,
+                           int32_t* tiles, int32_t max_tiles, void* stream) {
+  static_assert(FLUX_TILE_MASKED == flux::kTilePlanMasked, "tile-plan flag");
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!fa_mask || !seq_len || !tiles) return FLUX_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= cfg->n_layers) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || capacity < 1 || n_q < 0 || n_q > capacity)
+    return FLUX_ERR_INVALID_ARG;
+  if (max_tiles < (capacity + 127) / 128) return FLUX_ERR_INVALID_ARG;
+  if (n_q == 0) return FLUX_OK;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  return flux::cuda_status(flux::launch_prefill_tile_plan(
+      flux::geom_of(cfg), layer, fa_mask, seq_len, batch, capacity, n_q, tiles, max_tiles, status,
+      static_cast<cudaStream_t>(stream)));
 }
 
 int flux_sa_block_ranges(const flux_attn_cfg* cfg, int32_t n_qblocks, int32_t* ranges,

@@ -2,8 +2,10 @@
 //
 // * SA visibility arithmetic: the key-block ranges of the streaming pattern (sink
 //   blocks plus a local window of blocks, Table 6 / Figure 1 of the Flux Attention
-//   paper), used by the prefill tile scheduler, the decode split planner and
-//   flux_sa_block_ranges alike, so that one function defines the block indices.
+//   paper).  sa_key_blocks is the one definition of the block indices; every other
+//   use goes through it: visible_key_ranges (one query row: the decode split planner
+//   and the prefill per-key mask), visible_key_ranges_rows (the union over a tile of
+//   query rows: the prefill tile scheduler and its mask test) and flux_sa_block_ranges.
 // * mbarrier / bulk-copy wrappers (inline PTX) with bounded waits: a wait that runs
 //   past its time limit records FLUX_DEVICE_TIMEOUT in the status word and returns
 //   false instead of spinning forever or trapping.
@@ -69,6 +71,25 @@ __host__ __device__ __forceinline__ KeyRanges visible_key_ranges(int t, bool fa,
   r.hi0 = br.sink_end * block;
   r.lo1 = br.win_begin * block;
   r.hi1 = t + 1;
+  return r;
+}
+
+// Visible keys of the query rows [t_min, t_max] taken together, as
+// [0, hi0) U [lo1, t_max + 1).  Every key j in [t_min, t_max] is visible from row j
+// itself (its own block is in its window), so only keys below t_min need a rule: the
+// window start of a row never decreases with t, and a row whose window reaches back to
+// the sink (lo1 == 0) makes every earlier row do the same, so the union is the first
+// row's window joined with the last row's sink range.
+__host__ __device__ __forceinline__ KeyRanges visible_key_ranges_rows(int t_min, int t_max, bool fa,
+                                                                      int block, int sink,
+                                                                      int window) {
+  const KeyRanges first = visible_key_ranges(t_min, fa, block, sink, window);
+  const KeyRanges last = visible_key_ranges(t_max, fa, block, sink, window);
+  KeyRanges r;
+  r.lo0 = 0;
+  r.hi0 = first.lo1 == 0 ? 0 : last.hi0;
+  r.lo1 = first.lo1;
+  r.hi1 = t_max + 1;
   return r;
 }
 

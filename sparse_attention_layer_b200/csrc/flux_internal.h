@@ -86,6 +86,14 @@ cudaError_t launch_prefill(const AttnGeom& g, int layer, const uint32_t* fa_mask
                            const int32_t* seq_len, int batch, int capacity, int n_q, uint16_t* o,
                            unsigned* status, cudaStream_t stream);
 
+// The KV tiles flux_prefill visits per query tile (flux_prefill_tile_plan); entries
+// carry kTilePlanMasked when the kernel masks keys of the tile.
+constexpr unsigned kTilePlanMasked = 0x40000000u;
+cudaError_t launch_prefill_tile_plan(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                                     const int32_t* seq_len, int batch, int capacity, int n_q,
+                                     int32_t* tiles, int max_tiles, unsigned* status,
+                                     cudaStream_t stream);
+
 // ----- SA block ranges (the block indices the kernels use)
 cudaError_t launch_sa_block_ranges(const AttnGeom& g, int n_qblocks, int32_t* ranges,
                                    cudaStream_t stream);

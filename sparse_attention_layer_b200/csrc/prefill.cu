@@ -237,37 +237,28 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 
 // KV tiles of one query tile: tile index j < n0 is key tile j (the sink tiles); the
 // rest are key tiles w0 + (j - n0) (the window, up to the diagonal).  For FA n0 = 0
-// and w0 = 0.
+// and w0 = 0.  Built from the union of the tile's rows' visible keys
+// (visible_key_ranges_rows, the shared SA definition), rounded out to whole tiles: a
+// tile is visited iff it holds a key that some row of the query tile sees.
 struct TilePlan {
   int n0, w0, n_tiles;
   int t_min, t_max;   // absolute positions of the tile's first and last real query
-  int win_lo_tmax;    // first window key of the last query (SA)
-  bool fa;
+  int gap0, gap1;     // keys [gap0, gap1) are hidden from the last row (empty for FA)
 };
-
-__device__ __forceinline__ int window_lo(int t, int block, int window) {
-  const int w = (t / block - window / block + 1) * block;
-  return w > 0 ? w : 0;
-}
 
 __device__ __forceinline__ TilePlan plan_tiles(const PrefillArgs& a, bool fa, int t_min, int t_max) {
   TilePlan p;
-  p.fa = fa;
   p.t_min = t_min;
   p.t_max = t_max;
   const int last = t_max / BN;
-  p.win_lo_tmax = window_lo(t_max, a.block, a.window);
-  if (fa) {
-    p.n0 = 0;
-    p.w0 = 0;
-    p.n_tiles = last + 1;
-    return p;
-  }
-  // union over the tile's queries: [0, min(sink, t_max+1)) U [window_lo(t_min), t_max]
-  const int sink_hi = a.sink < t_max + 1 ? a.sink : t_max + 1;
-  const int n_sink_tiles = (sink_hi + BN - 1) / BN;
-  const int w0 = window_lo(t_min, a.block, a.window) / BN;
-  if (w0 <= n_sink_tiles) {
+  const KeyRanges u = visible_key_ranges_rows(t_min, t_max, fa, a.block, a.sink, a.window);
+  // The rows' sink/window gaps grow with t, so the last row's gap covers every row's.
+  const KeyRanges lr = visible_key_ranges(t_max, fa, a.block, a.sink, a.window);
+  p.gap0 = lr.hi0;
+  p.gap1 = lr.lo1;
+  const int n_sink_tiles = (u.hi0 + BN - 1) / BN;
+  const int w0 = u.lo1 / BN;
+  if (w0 <= n_sink_tiles) {  // FA, or the window reaches back to the sink tiles
     p.n0 = 0;
     p.w0 = 0;
     p.n_tiles = last + 1;
@@ -283,12 +274,24 @@ __device__ __forceinline__ int tile_key0(const TilePlan& p, int j) {
   return (j < p.n0 ? j : p.w0 + (j - p.n0)) * BN;
 }
 
-// True when some (query, key) pair of the tile is not visible.
-__device__ __forceinline__ bool tile_needs_mask(const TilePlan& p, int k0, int sink) {
-  if (k0 + BN - 1 > p.t_min) return true;  // crosses the causal diagonal / valid length
-  if (p.fa) return false;
-  if (k0 + BN <= sink) return false;       // wholly inside the sink
-  return k0 < p.win_lo_tmax;               // not wholly inside every query's window
+// True when some (query, key) pair of the tile is not visible: a key past the first
+// row (causal diagonal, valid length), or a key in the last row's sink/window gap.
+__device__ __forceinline__ bool tile_needs_mask(const TilePlan& p, int k0) {
+  if (k0 + BN - 1 > p.t_min) return true;
+  return k0 < p.gap1 && k0 + BN > p.gap0;
+}
+
+// The plan of query tile m_tile of sequence b, as the prefill kernel computes it.
+// ok = false for a sequence whose length is out of range (nothing is computed).
+__device__ __forceinline__ TilePlan plan_for(const PrefillArgs& a, int b, int m_tile, int& rows,
+                                             int& q_start, bool& ok) {
+  const int seq = a.seq_len[b];
+  ok = seq >= a.n_q && seq <= a.capacity;
+  q_start = seq - a.n_q;
+  const int row0 = m_tile * BM;
+  rows = min(BM, a.n_q - row0);
+  const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
+  return plan_tiles(a, fa, q_start + row0, q_start + row0 + rows - 1);
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -337,16 +340,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = blockIdx.z;
   const int kvh = h / (a.hq / a.hkv);
 
-  const int seq = a.seq_len[b];
-  if (seq < a.n_q || seq > a.capacity) {
+  int rows, q_start;
+  bool len_ok;
+  const TilePlan plan = plan_for(a, b, m_tile, rows, q_start, len_ok);
+  if (!len_ok) {
     if (tid == 0 && h == 0 && blockIdx.y == 0) atomicOr(a.status, kStatusBadLength);
     return;
   }
-  const int q_start = seq - a.n_q;
+  const int seq = q_start + a.n_q;
   const int row0 = m_tile * BM;                    // first query index of the tile
-  const int rows = min(BM, a.n_q - row0);
   const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
-  const TilePlan plan = plan_tiles(a, fa, q_start + row0, q_start + row0 + rows - 1);
 
   // The K producer thread initialises the barriers and issues the Q tile and the first
   // K tiles at once, while the MMA warp allocates tensor memory: the loads are in
@@ -506,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (warp & 3) * 32 + lane;         // query row within the tile
     const bool real_row = r < rows;
     const int t = plan.t_min + (real_row ? r : rows - 1);
-    const int wl = window_lo(t, a.block, a.window);
+    // this row's visible keys: [0, vr.hi0) U [vr.lo1, t], the shared SA definition
+    const KeyRanges vr = visible_key_ranges(t, fa, a.block, a.sink, a.window);
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t srow = tmem + g * 128 + lane_base;
     const uint32_t orow = tmem + kTmemO + g * 128 + lane_base;
@@ -520,15 +524,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bar_sfull + 8 * g, (j >> 1) & 1, a.status)) { ok = false; break; }
       tc_fence_after();
       const int k0 = tile_key0(plan, j);
-      const bool masked = tile_needs_mask(plan, k0, a.sink);
+      const bool masked = tile_needs_mask(plan, k0);
       // This row's visible key offsets i in [0, BN) of the tile: causal i <= lim, and for
       // SA outside the gap [gap0, gap1) between the sink and the window (has_gap: the
       // gap meets this tile).  The mask costs instructions on every key of a masked tile
       // (the diagonal tile of every causal row block), so the common causal-only case is
       // one compare and one select per key.
       const int lim = t - k0;
-      const int gap0 = plan.fa ? BN : min(max(a.sink - k0, 0), BN);
-      const int gap1 = plan.fa ? BN : min(max(wl - k0, 0), BN);
+      const int gap0 = min(max(vr.hi0 - k0, 0), BN);
+      const int gap1 = min(max(vr.lo1 - k0, 0), BN);
       const bool has_gap = __any_sync(0xffffffffu, gap0 < gap1);
       // Load 64 columns of the S row into s[] and apply the tile's mask.
       auto load_half = [&](uint32_t (&s)[64], int half) {
@@ -746,6 +750,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ tile schedule query
+
+// The KV tiles the prefill kernel visits for every query tile, computed by the same
+// plan_for / tile_needs_mask calls the kernel makes (flux_prefill_tile_plan).
+__global__ void __launch_bounds__(128) prefill_tile_plan_kernel(const PrefillArgs a, int32_t* tiles,
+                                                                int max_tiles) {
+  const int m_tile = blockIdx.x, b = blockIdx.y;
+  int rows, q_start;
+  bool ok;
+  const TilePlan p = plan_for(a, b, m_tile, rows, q_start, ok);
+  int32_t* out = tiles + (size_t(b) * a.n_mtiles + m_tile) * max_tiles;
+  for (int i = threadIdx.x; i < max_tiles; i += blockDim.x) {
+    int v = -1;
+    if (ok && i < p.n_tiles) {
+      const int k0 = tile_key0(p, i);
+      v = (k0 / BN) | (tile_needs_mask(p, k0) ? int(kTilePlanMasked) : 0);
+    }
+    out[i] = v;
+  }
+  if (!ok && threadIdx.x == 0 && m_tile == 0) atomicOr(a.status, kStatusBadLength);
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -753,16 +779,20 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encode_fn() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<EncodeTiledFn>(p);
+  return nullptr;
+}
+
+// The driver's tensor-map encoder, looked up once (a function-local static is
+// initialised once even when host threads race on the first call).
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  static const EncodeTiledFn fn = lookup_encode_fn();
   return fn;
 }
 
@@ -802,12 +832,9 @@ cudaError_t launch_prefill_t(const AttnGeom& g, const PrefillArgs& a, const uint
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_prefill(const AttnGeom& g, int layer, const uint32_t* fa_mask,
-                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
-                           const int32_t* seq_len, int batch, int capacity, int n_q, uint16_t* o,
-                           unsigned* status, cudaStream_t stream) {
+PrefillArgs prefill_args(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                         const int32_t* seq_len, int capacity, int n_q, uint16_t* o,
+                         unsigned* status) {
   PrefillArgs a;
   a.fa_mask = fa_mask;
   a.mask_words = g.mask_words;
@@ -824,10 +851,30 @@ cudaError_t launch_prefill(const AttnGeom& g, int layer, const uint32_t* fa_mask
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(g.head_dim)));
   a.o = o;
   a.status = status;
+  return a;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                           const int32_t* seq_len, int batch, int capacity, int n_q, uint16_t* o,
+                           unsigned* status, cudaStream_t stream) {
+  const PrefillArgs a = prefill_args(g, layer, fa_mask, seq_len, capacity, n_q, o, status);
   if (a.n_mtiles > 65535) return cudaErrorInvalidValue;
   if (g.head_dim == 128) return launch_prefill_t<128>(g, a, q, k_cache, v_cache, batch, stream);
   if (g.head_dim == 64) return launch_prefill_t<64>(g, a, q, k_cache, v_cache, batch, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_tile_plan(const AttnGeom& g, int layer, const uint32_t* fa_mask,
+                                     const int32_t* seq_len, int batch, int capacity, int n_q,
+                                     int32_t* tiles, int max_tiles, unsigned* status,
+                                     cudaStream_t stream) {
+  const PrefillArgs a = prefill_args(g, layer, fa_mask, seq_len, capacity, n_q, nullptr, status);
+  if (a.n_mtiles > 65535) return cudaErrorInvalidValue;
+  prefill_tile_plan_kernel<<<dim3(a.n_mtiles, batch), 128, 0, stream>>>(a, tiles, max_tiles);
+  return cudaGetLastError();
 }
 
 }  // namespace flux

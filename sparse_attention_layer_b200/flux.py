@@ -37,8 +37,11 @@ EXPORTED = (
     "flux_decode_workspace_size", "flux_decode", "flux_sa_block_ranges",
     "flux_get_device_status", "flux_status_string", "flux_version", "flux_decode_static",
     "flux_kv_compact_ring", "flux_kv_append_ring", "flux_decode_ring",
-    "flux_selftest_wait_timeout",
+    "flux_selftest_wait_timeout", "flux_prefill_tile_plan",
 )
+
+# flag bit of a flux_prefill_tile_plan entry: the kernel masks keys of that tile
+FLUX_TILE_MASKED = 0x40000000
 
 # bytes of the scratch array flux_decode_static keeps inside the library
 FLUX_DECODE_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -136,6 +139,9 @@ def lib() -> ctypes.CDLL:
         L.flux_decode_ring.restype = ctypes.c_int
         L.flux_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         L.flux_selftest_wait_timeout.restype = ctypes.c_int
+        L.flux_prefill_tile_plan.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, i32, i32,
+                                             i32, vp, i32, vp]
+        L.flux_prefill_tile_plan.restype = ctypes.c_int
         L.flux_sa_block_ranges.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp]
         L.flux_sa_block_ranges.restype = ctypes.c_int
         _lib = L
@@ -352,3 +358,19 @@ def flux_sa_block_ranges(cfg: AttnCfg, n_qblocks: int, ranges, stream=None) -> N
         ctypes.byref(c), int(n_qblocks), _ptr(ranges, "ranges", torch.int32, (n_qblocks, 3)),
         _stream(stream))
     _check("flux_sa_block_ranges", st)
+
+
+def flux_prefill_tile_plan(cfg: AttnCfg, layer: int, fa_mask, seq_len, capacity: int, n_q: int,
+                           tiles, stream=None) -> None:
+    """The KV tiles flux_prefill visits: tiles [B][ceil(n_q/128)][max_tiles] int32 gets
+    the 128-key tile index of each visited tile (| FLUX_TILE_MASKED where the kernel
+    masks keys), -1 after the last."""
+    batch = seq_len.shape[0]
+    n_mt = (n_q + 127) // 128
+    max_tiles = tiles.shape[2]
+    c = cfg.c()
+    st = lib().flux_prefill_tile_plan(
+        ctypes.byref(c), int(layer), _ptr(fa_mask, "fa_mask", torch.int32, (batch, cfg.mask_words)),
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, int(capacity), int(n_q),
+        _ptr(tiles, "tiles", torch.int32, (batch, n_mt, max_tiles)), max_tiles, _stream(stream))
+    _check("flux_prefill_tile_plan", st)

@@ -184,6 +184,29 @@ def check_sa_key_blocks(orc):
             assert got == want, (block, qb, sorted(got), sorted(want))
 
 
+def check_key_tiles_of_rows(orc):
+    """Key tiles visited / masked for a run of query rows: the FA closed form (tiles up to
+    the last row's, masked where a key passes the first row), agreement with the key-block
+    sets of whole query blocks when tile == block, and two hand-worked SA examples."""
+    for t_min, t_max, tile in ((0, 127, 128), (1000, 1127, 128), (5, 5, 64), (300, 427, 64)):
+        vis, msk = orc.key_tiles_of_rows(True, np.arange(t_min, t_max + 1), tile, 64, 64, 256)
+        assert vis == list(range(t_max // tile + 1))
+        assert msk == [kt for kt in vis if kt * tile + tile - 1 > t_min]
+    for block, sink, window in ((64, 64, 256), (128, 128, 2048), (64, 0, 64)):
+        for qb in (0, 1, 3, 7, 20, 33):
+            rows = np.arange(qb * block, (qb + 1) * block)
+            vis, _ = orc.key_tiles_of_rows(False, rows, block, block, sink, window)
+            assert set(vis) == orc.sa_visible_key_blocks(qb, qb + 1, block, sink, window)
+    # block 64, sink 128, window 256, rows 1000..1127, 128-key tiles: sink keys [0, 128),
+    # row 1000 sees from key 768 (block 12), row 1127 from key 896 (block 14)
+    assert orc.key_tiles_of_rows(False, np.arange(1000, 1128), 128, 64, 128, 256) == \
+        ([0, 6, 7, 8], [6, 7, 8])
+    # block 64, sink 64, window 128: sink keys [0, 64) (keys 64..127 of tile 0 hidden),
+    # row 1000 sees from key 896, row 1127 from key 1024
+    assert orc.key_tiles_of_rows(False, np.arange(1000, 1128), 128, 64, 64, 128) == \
+        ([0, 7, 8], [0, 7, 8])
+
+
 # ---------------------------------------------------------------- decode, append
 
 
@@ -319,7 +342,8 @@ def check_ring_placement_hand_example(orc):
 ALL_CHECKS = [
     check_attention_vs_library, check_attention_closed_forms, check_softmax_rows,
     check_sa_counts_golden, check_sa_count_closed_form, check_sa_covers_fa,
-    check_sa_token_reading_close, check_sa_key_blocks, check_decode_is_prefill_row,
+    check_sa_token_reading_close, check_sa_key_blocks, check_key_tiles_of_rows,
+    check_decode_is_prefill_row,
     check_kv_append, check_router_golden, check_pool_indices, check_omega_pages,
     check_router_error_bound, check_ring_keeps_every_visible_key,
     check_ring_placement_hand_example,

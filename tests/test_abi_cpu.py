@@ -145,3 +145,21 @@ def test_product_package_never_imports_the_oracle():
             if fn.endswith(".py"):
                 with open(os.path.join(dirpath, fn)) as f:
                     assert not pat.search(f.read()), f"{fn} imports the oracle"
+
+
+def test_tile_plan_flag_and_host_checks(L):
+    with open(os.path.join(ROOT, "include", "flux.h")) as f:
+        text = f.read()
+    assert int(re.search(r"#define FLUX_TILE_MASKED (0x[0-9a-fA-F]+)", text).group(1), 16) == \
+        flux.FLUX_TILE_MASKED
+    c = _cfg()
+    fake = ctypes.c_void_p(1 << 20)
+    # max_tiles must cover ceil(capacity / 128) key tiles
+    assert L.flux_prefill_tile_plan(ctypes.byref(c), 0, fake, fake, 1, 1024, 512, fake, 7,
+                                    None) == flux.FLUX_ERR_INVALID_ARG
+    assert L.flux_prefill_tile_plan(ctypes.byref(c), 0, fake, fake, 1, 1024, 2048, fake, 8,
+                                    None) == flux.FLUX_ERR_INVALID_ARG   # n_q > capacity
+    assert L.flux_prefill_tile_plan(ctypes.byref(c), 40, fake, fake, 1, 1024, 512, fake, 8,
+                                    None) == flux.FLUX_ERR_INVALID_ARG   # layer out of range
+    assert L.flux_prefill_tile_plan(ctypes.byref(c), 0, fake, fake, 1, 1024, 0, fake, 8,
+                                    None) == flux.FLUX_OK                # nothing to plan

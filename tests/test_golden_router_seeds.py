@@ -22,3 +22,14 @@ def test_llama_router_seed_reproduces():
     for key in ("router_seed", "n_sa_layers", "omega_msr", "pooled_tokens", "fa_bits"):
         assert got[key] == want[key], key
     assert got["min_margin_over_fp64_bound"] > 1000.0
+
+
+def test_workload_seed_constants_match_the_record():
+    """The workload definitions carry the recorded seeds as constants (the product
+    package never reads the test tree)."""
+    from sparse_attention_layer_b200 import configs
+    with open(os.path.join(ROOT, "tests", "golden", "router_seeds.json")) as f:
+        rec = json.load(f)
+    for w in (configs.LLAMA_PREFILL, configs.QWEN_PREFILL):
+        assert w.router_seed == rec[w.name]["router_seed"], w.name
+        assert w.target_sa_layers == rec[w.name]["n_sa_layers"], w.name

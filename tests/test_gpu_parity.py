@@ -129,6 +129,75 @@ def test_sa_block_ranges_exact(block, sink, window):
         assert got == want, (qb, r[qb].tolist(), sorted(want))
 
 
+def _tile_plan(cfg, layer, mask, seq_len, capacity, n_q):
+    n_mt = (n_q + 127) // 128
+    max_tiles = (capacity + 127) // 128
+    tiles = torch.empty(len(seq_len), n_mt, max_tiles, dtype=torch.int32, device="cuda")
+    seq = torch.tensor(seq_len, dtype=torch.int32, device="cuda")
+    flux.flux_prefill_tile_plan(cfg, layer, mask, seq, capacity, n_q, tiles)
+    torch.cuda.synchronize()
+    assert flux.flux_get_device_status() == 0
+    return tiles.cpu().numpy()
+
+
+def _check_tile_plan(cfg, tiles, b, m, q_start, n_q, fa):
+    """Query tile m of sequence b: the kernel's visited tiles (in visiting order) and the
+    ones it masks equal the oracle's sets from the dense visibility mask."""
+    rows = q_start + np.arange(m * 128, min(n_q, (m + 1) * 128))
+    want_vis, want_msk = orc.key_tiles_of_rows(fa, rows, 128, cfg.block, cfg.sink, cfg.window)
+    row = tiles[b, m]
+    n = int((row >= 0).sum())
+    assert (row[n:] == -1).all() and (row[:n] >= 0).all()
+    got = row[:n]
+    got_vis = (got & ~flux.FLUX_TILE_MASKED).tolist()
+    got_msk = [int(e & ~flux.FLUX_TILE_MASKED) for e in got if e & flux.FLUX_TILE_MASKED]
+    assert got_vis == want_vis, (b, m, got_vis, want_vis)
+    assert got_msk == want_msk, (b, m, got_msk, want_msk)
+
+
+@pytest.mark.parametrize("block,sink,window", [
+    (64, 0, 64), (64, 64, 256), (64, 128, 256), (64, 128, 2048), (64, 128, 4096),
+    (128, 0, 128), (128, 128, 128), (128, 128, 2048), (128, 256, 1024), (128, 128, 4096)])
+def test_prefill_tile_plan_exact(block, sink, window):
+    """SA block indices of the prefill kernel, exactly: the 128-key tiles it visits for
+    every 128-query tile, and the tiles it masks, equal the oracle's (tiles holding a key
+    some row of the query tile sees; of those, tiles with a pair some row does not see).
+    One-shot and chunked prompts (queries after a prefix), ragged last tile, per-sequence
+    routes in one batch."""
+    cfg = AttnCfg(2, 8, 2, 128, block, sink, window)
+    n_q = 3000                                  # 23 full query tiles + 56 rows
+    q_starts = [0, 77, 4096, 5000]
+    seq_len = [qs + n_q for qs in q_starts]
+    capacity = max(seq_len) + 5
+    fa_rows = [[], [0], [1], []]                # layer 0: SA, FA, SA, SA; layer 1: SA, SA, FA, SA
+    mask = mask_words(len(seq_len), cfg.n_layers, fa_rows).cuda()
+    for layer in (0, 1):
+        tiles = _tile_plan(cfg, layer, mask, seq_len, capacity, n_q)
+        for b, qs in enumerate(q_starts):
+            for m in range(tiles.shape[1]):
+                _check_tile_plan(cfg, tiles, b, m, qs, n_q, layer in fa_rows[b])
+
+
+@pytest.mark.parametrize("name", ["llama31_8b_prefill_8k", "qwen3_4b_prefill_128k"])
+def test_prefill_tile_plan_full_size(name):
+    """The full-size prompts' tile schedules, exactly, for the SA route on every query tile
+    of the Llama prompt and on sampled query tiles of the 131072-token Qwen prompt (the FA
+    route checked on sampled tiles)."""
+    w = configs.ALL[name]
+    cfg = cfg_of(w)
+    for fa in (False, True):
+        mask = mask_words(1, cfg.n_layers, [[3] if fa else []]).cuda()
+        tiles = _tile_plan(cfg, 3, mask, [w.seq], w.seq, w.seq)
+        n_mt = tiles.shape[1]
+        if n_mt <= 64 and not fa:
+            ms = range(n_mt)
+        else:
+            g = np.random.default_rng(7)
+            ms = sorted({0, 1, 15, 16, 17, 31, 32, 33, n_mt - 1} | set(g.integers(0, n_mt, 12).tolist()))
+        for m in ms:
+            _check_tile_plan(cfg, tiles, 0, m, 0, w.seq, fa)
+
+
 # ------------------------------------------------------------------------ KV append
 
 
@@ -315,6 +384,40 @@ def test_decode_llama_full_size():
     ctx = [w.seq] * w.batch
     _decode_case(cfg, ctx, [True] * w.batch, 1, seed=1000, capacity=w.capacity(), layer=3)
     _decode_case(cfg, ctx, [False] * w.batch, 2, seed=1001, capacity=w.capacity(), layer=4)
+
+
+@pytest.mark.parametrize("fa", [True, False])
+def test_decode_llama_batch1_128k(fa):
+    """Llama-3.1-8B heads, one sequence at a 131072-token context (the sweep's longest
+    point at batch 1): the 8 (sequence, KV head) pairs are each cut over ~18 CTAs."""
+    cfg = AttnCfg(32, 32, 8, 128, 128, 128, 2048)
+    _decode_case(cfg, [131072], [fa], 2, seed=1200 + fa, layer=9)
+
+
+def test_decode_split_cap_single_pair():
+    """One KV head, 8 query heads, a 131072-token FA context and SA beside it: a single
+    pair of 1025 stages is dealt to ~61 CTAs, the most the split planner allows."""
+    cfg = AttnCfg(1, 8, 1, 128, 128, 128, 2048)
+    _decode_case(cfg, [131072, 131000], [True, False], 1, seed=1210)
+
+
+def test_decode_llama_batch32_32k():
+    """Llama-3.1-8B decode at the sweep's batch 32 x 32768 context, mixed routes."""
+    cfg = AttnCfg(32, 32, 8, 128, 128, 128, 2048)
+    ctx = [32768] * 32
+    fa = [b % 2 == 0 for b in range(32)]
+    _decode_case(cfg, ctx, fa, 1, seed=1220, layer=17)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_pages_sa_geometry(d):
+    """The pages' SA kernel geometry (Table 6: block 64, sink 128) with a 2048-token
+    window, Llama heads, head_dim 64 and 128: 16 sequences at a 32768-token context,
+    SA and FA sequences in one batch, across a block boundary."""
+    cfg = AttnCfg(32, 32, 8, d, 64, 128, 2048)
+    ctx = [32768 - 2] * 8 + [32768 + 61] * 8
+    fa = [b % 4 == 0 for b in range(16)]
+    _decode_case(cfg, ctx, fa, 3, seed=1230 + d, layer=5)
 
 
 def test_decode_graph_replay_matches_eager():

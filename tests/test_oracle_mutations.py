@@ -35,6 +35,9 @@ MUTATIONS = {
                           "k_out[b, :, start + i + 1, :] = k_new[b, i]"),
     "append_no_advance": ("len_out[b] = start + n_new", "len_out[b] = start"),
     "ring_slot_offset": ("sink + (p - sink) % ring_rows)", "(p - sink) % ring_rows)"),
+    "tile_mask_never": ("if not per_tile[:, kt, :].all()]", "if not per_tile[:, kt, :].any()]"),
+    "tile_visit_misses_last": ("n_tiles = int(q_pos.max()) // tile + 1",
+                               "n_tiles = int(q_pos.max()) // tile"),
     "ring_keeps_too_few": ("np.arange(max(sink, seq_len - ring_rows), seq_len",
                            "np.arange(max(sink, seq_len - ring_rows + 1), seq_len"),
 }
