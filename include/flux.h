@@ -15,12 +15,13 @@
  *                   local window of KV blocks; Table 6, Figure 1 caption), chosen on
  *                   the device from the layer's bit in the routing mask.
  *   flux_decode     one autoregressive step of the same attention over the cache
- *                   (split-KV partial softmax plus a combine pass).
+ *                   (split-KV partial softmax, merged by the last CTA of each split);
+ *                   flux_decode_append also appends the step's new K/V row.
  *
  * Conventions shared by every call
  *   - Every pointer argument that names tensor data is a DEVICE pointer owned by the
  *     caller.  The library allocates and frees nothing; scratch space (the decode
- *     workspace) is passed in by the caller.
+ *     workspace, zero-filled once by the caller) is passed in by the caller.
  *   - bf16 tensors are passed as uint16_t (raw bf16 bit patterns), row-major, densely
  *     packed, with the layouts stated per call.  Base pointers must be 16-byte aligned.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
@@ -147,7 +148,8 @@ int flux_prefill(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mas
                  const int32_t* seq_len, int32_t batch, int32_t capacity, int32_t n_q,
                  uint16_t* o, void* stream);
 
-/* Bytes of device workspace flux_decode needs for this geometry and batch. */
+/* Bytes of device workspace flux_decode needs for this geometry and batch: arrival
+ * counters at fixed offsets (4352 bytes), then split partial results. */
 size_t flux_decode_workspace_size(const flux_attn_cfg* cfg, int32_t batch);
 
 /*
@@ -155,16 +157,43 @@ size_t flux_decode_workspace_size(const flux_attn_cfg* cfg, int32_t batch);
  * reused), after the new token's K/V row has been appended.
  *   q   [batch][n_q_heads][head_dim] bf16, the query at position seq_len[b] - 1.
  *   o   [batch][n_q_heads][head_dim] bf16, written.
- *   workspace  caller-owned device buffer of >= flux_decode_workspace_size() bytes
- *              (split partial results; contents need no initialisation).
- * Split-KV kernel (bulk-copy pipeline, 128-bit shared loads, warp-shuffle
- * reductions) plus a combine kernel.  SA reads only the sink and window rows.
+ *   workspace  caller-owned device buffer of >= flux_decode_workspace_size() bytes,
+ *              ZERO-FILLED ONCE before its first use (cudaMemset): its arrival
+ *              counters must start at zero, and every call leaves them at zero, so one
+ *              workspace serves any later call of any geometry that fits it.  Calls
+ *              that share a workspace must not overlap on the GPU.  After a call that
+ *              reported FLUX_DEVICE_TIMEOUT, zero it again.
+ * One kernel launch (programmatic dependent launch, so it may start while the
+ * previous kernel on the stream drains): a persistent split-KV kernel (bulk-copy
+ * pipeline, 128-bit shared loads, warp-shuffle reductions); the CTA that finishes a
+ * split pair merges its partial results.  SA reads only the sink and window rows.
  * seq_len[b] == 0 writes zeros; seq_len[b] > capacity sets FLUX_DEVICE_BAD_LENGTH.
  */
 int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
                 const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
                 const int32_t* seq_len, int32_t batch, int32_t capacity, uint16_t* o,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * flux_decode_append -- flux_kv_append of one new row per sequence followed by
+ * flux_decode, in one kernel launch (the decode step of one layer: Table 3's decode
+ * reusing the prefill route, over the persistent KV cache of Tables 15/16).
+ *   k_new, v_new  [batch][1][n_kv_heads][head_dim] bf16, the step's new key and value.
+ *   k_cache, v_cache, seq_len  read and written: for every sequence with room
+ *                  (seq_len[b] < capacity) the new row is written at position
+ *                  seq_len[b] and seq_len[b] is advanced by one, exactly as
+ *                  flux_kv_append would; the query q[b] sits at the new row's position.
+ *   o, workspace   as for flux_decode.
+ * Results equal flux_kv_append + flux_decode bit for bit (same keys, same split plan,
+ * same arithmetic: the new key is streamed from k_new instead of the cache).  A
+ * sequence without room writes zeros, keeps its rows and length and sets
+ * FLUX_DEVICE_CAPACITY.
+ */
+int flux_decode_append(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                       const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                       uint16_t* k_cache, uint16_t* v_cache, int32_t* seq_len, int32_t batch,
+                       int32_t capacity, uint16_t* o, void* workspace, size_t workspace_bytes,
+                       void* stream);
 
 /* Size of the scratch array flux_decode_static keeps inside the library (32 MiB). */
 #define FLUX_DECODE_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
@@ -190,8 +219,9 @@ int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask
  *   allocation is still allowed, and before any stream capture.
  *   All calls share the one array, so calls that can overlap on the GPU (different
  *   streams, or devices sharing a context) race and corrupt each other's results;
- *   serialise them.  The array keeps the last call's contents; nothing in it needs to
- *   start at zero, because every record the combine pass reads is written first.
+ *   serialise them.  The array keeps the last call's contents.  Only its arrival
+ *   counters must start at zero: the array is zeroed when the module loads, every call
+ *   leaves them at zero, and the partial records are written before they are read.
  */
 int flux_decode_static(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
                        const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
@@ -233,6 +263,16 @@ int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa
                      const uint16_t* q, const uint16_t* k_ring, const uint16_t* v_ring,
                      const int32_t* seq_len, int32_t batch, int32_t ring_rows, uint16_t* o,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* flux_decode_append_ring -- flux_kv_append_ring of one new row per sequence followed
+ * by flux_decode_ring, in one kernel launch; results equal the two calls bit for bit.
+ * A sequence routed to FA writes zeros, is not appended and sets
+ * FLUX_DEVICE_RING_ROUTE. */
+int flux_decode_append_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                            const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                            uint16_t* k_ring, uint16_t* v_ring, int32_t* seq_len, int32_t batch,
+                            int32_t ring_rows, uint16_t* o, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /*
  * flux_sa_block_ranges -- the SA key-block set of each query block, as the kernels

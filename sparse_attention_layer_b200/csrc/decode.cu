@@ -3,26 +3,39 @@
 //
 // One query token per sequence attends the keys of its route: FA reads the whole
 // cache [0, seq_len), SA reads only the sink rows and the window rows.  Decode is
-// bound by HBM bandwidth, so the kernel is built around moving K/V bytes:
+// bound by HBM bandwidth, so the kernel is built around moving K/V bytes, and one
+// call is one kernel launch:
 //
 //  * the visible keys of each (sequence, KV head) pair are cut into 128-key stages;
 //    all pairs' stages, laid end to end, are dealt to the persistent grid (one CTA
 //    per SM) as equal contiguous ranges, so every CTA streams the same number of
 //    stages (FA and SA pairs, ragged lengths alike) and closes a partial result only
 //    where its range crosses a pair boundary -- one to three times per CTA at large
-//    batch, instead of once per fixed-size split;
-//  * one producer lane streams each split's K and V rows -- contiguous in the
+//    batch, instead of once per fixed-size split.  When there are no more pairs than
+//    CTAs and streaming the longest pair whole costs less than splitting plus merging
+//    (a streaming-rate model, below), each CTA takes one pair whole instead;
+//  * one producer lane streams each piece's K and V rows -- contiguous in the
 //    [B][Hkv][cap][d] cache -- into a 3-stage ring of 128-key stages with 1-D bulk
 //    copies (cp.async.bulk, no cluster), completing on mbarriers; the group's query
-//    rows ride along with the first stage of every split;
+//    rows ride along with the first stage of every piece;
 //  * 8 consumer warps (16 keys each per stage) read the stage with 128-bit shared
 //    loads: 8 lanes cover one key row (16 B each), 4 rows per warp instruction, all
 //    G = Hq/Hkv query heads of the group at once, with packed fp32x2 FMAs; the q.k
 //    partial sums are reduced across the 8 lanes with a transposing butterfly (each
 //    level hands half of the remaining head sums to the partner lane);
 //  * online softmax in the log2 domain per head; P.V accumulates in fp32 registers;
-//  * each item writes (running max, running sum, unnormalised accumulator) per head
-//    to the caller's workspace; a combine kernel merges the splits and writes bf16.
+//  * a piece that covers its whole pair normalises and writes the bf16 output itself;
+//    the pieces of a split pair write (running max, running sum, unnormalised
+//    accumulator) per head to the workspace, and the CTA that finishes the pair's last
+//    piece (an arrival counter in the workspace) merges them and writes the output;
+//  * the appending variant (flux_decode_append) also takes the step's new K/V row:
+//    the pair's newest key is streamed from k_new / v_new instead of the cache, the
+//    CTA that holds it writes the row into the cache, and the last CTA to finish
+//    reading the lengths (a second arrival counter) advances seq_len.
+//
+// The arrival counters live at fixed offsets at the start of the workspace, so they
+// do not move with the geometry; every call leaves them at zero, and a workspace only
+// has to be zero-filled once, before its first call.
 #include <math.h>
 
 #include <mutex>
@@ -31,11 +44,13 @@
 #include "flux_device.cuh"
 #include "flux_internal.h"
 
-// Scratch for flux_decode_static: the split partials that flux_decode keeps in the
-// caller's workspace, held instead in a fixed array inside the library image.  Every
-// GPU that loads the library reserves these bytes until the process exits.  In host
-// code this name is only a host-side stand-in: its device address comes from
-// cudaGetSymbolAddress (see static_scratch_address below).
+// Scratch for flux_decode_static: the split partials and arrival counters that
+// flux_decode keeps in the caller's workspace, held instead in a fixed array inside
+// the library image.  Every GPU that loads the library reserves these bytes until the
+// process exits; like every __device__ array without an initialiser it starts zeroed,
+// which is the state the arrival counters need.  In host code this name is only a
+// host-side stand-in: its device address comes from cudaGetSymbolAddress (see
+// static_scratch_address below).
 static __device__ __align__(256) unsigned char g_decode_static_scratch[FLUX_DECODE_STATIC_SCRATCH_BYTES];
 
 namespace flux {
@@ -45,9 +60,11 @@ constexpr int kStageKeys = kDecStageKeys;
 constexpr int kMaxStages = 3;
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kKeysPerWarp = kStageKeys / kConsumerWarps;  // 16 keys per warp per stage
 constexpr int kPasses = kKeysPerWarp / 4;                  // 4 keys per warp instruction
 static_assert(kPasses == 4, "the tile maximum below is written for 4 passes");
+constexpr uint32_t kRouteFa = 0x80000000u;  // route bit of a per-sequence info word
 
 struct DecodeArgs {
   const uint32_t* fa_mask;
@@ -55,33 +72,33 @@ struct DecodeArgs {
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* v;
-  const int32_t* seq_len;
+  const uint16_t* k_new;  // appending variant: [B][1][Hkv][D]; otherwise null
+  const uint16_t* v_new;
+  int32_t* seq_len;       // written only by the appending variant
   int batch, capacity, hkv, block, sink, window;
   float scale_log2;  // log2(e) / sqrt(d)
   int ring_rows;     // 0: contiguous cache; > 0: SA ring cache of sink + ring_rows rows
   int rows;          // physical rows per (sequence, KV head)
+  unsigned* ws_ctr;  // [kDecCtaCounters] split-pair arrivals, then the length arrival
   float* ws_acc;     // [B][Hkv][kDecMaxSplits][G][D]
   float2* ws_ml;     // [B][Hkv][kDecMaxSplits][G] = (max, sum)
-  int* ws_nsplit;    // [B][Hkv]: partial results written for the pair
   uint16_t* o;
   unsigned* status;
 };
 
-// The visible keys of sequence b's decode query, flattened in position order and laid
-// out in up to three physically contiguous pieces: [0, len0) (sink, or everything in a
-// contiguous cache's merged case), then [start1, start1 + len1) and
-// [start2, start2 + len2) (the window; two pieces when it wraps around a ring cache).
+// The visible keys of a decode query at position T - 1 (T keys in the sequence,
+// counting the appended one), flattened in position order and laid out in up to three
+// physically contiguous pieces: [0, len0) (sink, or everything in a contiguous
+// cache's merged case), then [start1, start1 + len1) and [start2, start2 + len2) (the
+// window; two pieces when it wraps around a ring cache).
 struct Plan {
   int n_vis, stages;
   int len0, start1, len1, start2;
 };
 
-__device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
+__device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int T, bool fa) {
   Plan p{0, 0, 0, 0, 0, 0};
-  const int T = a.seq_len[b];
-  if (T <= 0 || T > a.capacity) return p;
-  const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
-  if (a.ring_rows > 0 && fa) return p;  // a ring cache only holds what SA reads
+  if (T <= 0) return p;
   const KeyRanges r = visible_key_ranges(T - 1, fa, a.block, a.sink, a.window);
   if (a.ring_rows == 0) {
     p.len0 = r.hi0 - r.lo0;
@@ -109,10 +126,17 @@ __device__ __forceinline__ Plan make_plan(const DecodeArgs& a, int b) {
   return p;
 }
 
+// Physical row of position t (the appended key's destination).
+__device__ __forceinline__ int physical_row(const DecodeArgs& a, int t) {
+  if (a.ring_rows == 0 || t < a.sink) return t;
+  return a.sink + (t - a.sink) % a.ring_rows;
+}
+
 // One CTA's piece of one pair: the pair's stages [k0, k1) (virtual keys [v0, v1)).
-// split numbers the CTAs that share the pair, n_split counts them.
+// split numbers the CTAs that share the pair, n_split counts them; first_cta is the
+// CTA holding split 0 (it indexes the pair's arrival counter).
 struct Item {
-  int b, kvh, split, n_split;
+  int b, kvh, split, n_split, first_cta;
   int v0, v1;
   int seg_end;  // global stage index where this piece ends
   Plan p;
@@ -128,9 +152,45 @@ __device__ __forceinline__ int stages_per_cta(int total, int max_pair_stages) {
   return max(1, max(even, cap));
 }
 
+// Streaming-rate model the planner uses to choose between two ways of dealing the
+// stages (constants measured on B200):
+//  * split: equal contiguous stage ranges over the whole grid (above); pairs longer
+//    than a range are cut, and their partial results are merged at the end;
+//  * whole pairs: CTA p streams pair p from first key to last and writes the final
+//    output itself; no partials, nothing to merge.
+// A stage costs stage_bytes / kHbmBytesPerNs for every CTA streaming at the same time
+// (HBM is shared), but at least stage_bytes / kCtaBytesPerNs (the rate one CTA's
+// consumer warps sustain on their own); merging split partials adds about kMergeNs
+// (partial writes, the arrival and the merging CTA's dependent reads).  Whole pairs
+// win when the longest pair streams, at that rate, in less time than the even split
+// plus the merge: e.g. 16 sequences at 32K context on the SA route (128 pairs of 17
+// stages), not on the FA route or at 8 sequences.
+constexpr float kHbmBytesPerNs = 6400.f;
+constexpr float kCtaBytesPerNs = 48.f;
+constexpr float kMergeNs = 3000.f;
+
+__device__ __forceinline__ bool whole_pairs_pay(int total, int max_pair_stages, int n_pairs,
+                                                int grid, float stage_bytes) {
+  if (n_pairs > grid || max_pair_stages == 0) return false;
+  const float solo = stage_bytes / kCtaBytesPerNs;
+  const float t_pairs =
+      float(max_pair_stages) * fmaxf(solo, float(n_pairs) * stage_bytes / kHbmBytesPerNs);
+  const int per = stages_per_cta(total, max_pair_stages);
+  const float t_split = float(per) * fmaxf(solo, float(grid) * stage_bytes / kHbmBytesPerNs) +
+                        (per < max_pair_stages ? kMergeNs : 0.f);
+  return t_pairs < t_split;
+}
+
+// Per-sequence word kept in shared memory: keys attended (T, counting an appended
+// key; 0 = nothing to attend) | kRouteFa.  The kernel reads seq_len from global memory
+// once, in its prologue: the appending variant rewrites it while the grid runs.
+__device__ __forceinline__ Plan plan_of(const DecodeArgs& a, uint32_t info) {
+  return make_plan(a, int(info & ~kRouteFa), (info & kRouteFa) != 0u);
+}
+
 // The piece that starts at global stage s of a range ending at end.
-__device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix, int s, int end,
-                                        int per) {
+__device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix,
+                                        const uint32_t* info, int s, int end, int per) {
   int lo = 0, hi = a.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -138,15 +198,16 @@ __device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix, 
   }
   Item it;
   it.b = lo;
-  it.p = make_plan(a, lo);
+  it.p = plan_of(a, info[lo]);
   const int ns = it.p.stages;
   const int r = s - prefix[lo];
   it.kvh = r / ns;
   const int pair0 = prefix[lo] + it.kvh * ns;
   const int pair1 = pair0 + ns;
   it.seg_end = min(end, pair1);
-  it.split = s / per - pair0 / per;
-  it.n_split = (pair1 - 1) / per - pair0 / per + 1;
+  it.first_cta = pair0 / per;
+  it.split = s / per - it.first_cta;
+  it.n_split = (pair1 - 1) / per - it.first_cta + 1;
   it.v0 = (s - pair0) * kDecStageKeys;
   it.v1 = min(it.p.n_vis, (it.seg_end - pair0) * kDecStageKeys);
   return it;
@@ -154,7 +215,8 @@ __device__ __forceinline__ Item item_at(const DecodeArgs& a, const int* prefix, 
 
 // Stages cover consecutive virtual keys of the item, whatever physical pieces they
 // come from, so a key's stage row (and hence the arithmetic) depends only on its place
-// in the position order: a ring cache and a contiguous cache give identical results.
+// in the position order: a ring cache and a contiguous cache give identical results,
+// and so do an appended key streamed from k_new and the same key read from the cache.
 __device__ __forceinline__ int item_stages(const Item& it) {
   return (it.v1 - it.v0 + kStageKeys - 1) / kStageKeys;
 }
@@ -163,11 +225,19 @@ __device__ __forceinline__ int stage_keys(const Item& it, int k) {
   return min(kStageKeys, it.v1 - it.v0 - k * kStageKeys);
 }
 
-// Physical runs of stage k: up to three (first physical row, count, stage row) triples.
-__device__ __forceinline__ int stage_runs(const Item& it, int k, int (&row)[3], int (&cnt)[3],
-                                          int (&dst)[3]) {
+// Physical runs of stage k: up to three (first physical row, count, stage row) triples
+// read from the cache.  With an appended key (the pair's last virtual key, position
+// T - 1) in the stage, that key is left out of the runs and new_dst is its stage row
+// (it comes from k_new / v_new); otherwise new_dst = -1.
+__device__ __forceinline__ int stage_runs(const Item& it, int k, bool append, int (&row)[3],
+                                          int (&cnt)[3], int (&dst)[3], int& new_dst) {
   const int vs = it.v0 + k * kStageKeys;
-  const int ve = min(it.v1, vs + kStageKeys);
+  int ve = min(it.v1, vs + kStageKeys);
+  new_dst = -1;
+  if (append && ve == it.p.n_vis) {
+    new_dst = ve - 1 - vs;
+    --ve;
+  }
   const int len2 = it.p.n_vis - it.p.len0 - it.p.len1;
   const int pvs[3] = {0, it.p.len0, it.p.len0 + it.p.len1};
   const int pln[3] = {it.p.len0, it.p.len1, len2};
@@ -260,24 +330,27 @@ struct DecodeSmemLayout {
   static constexpr size_t off_k = 0;
   static constexpr size_t off_v = off_k + kStages * kv_stage * 2;
   static constexpr size_t off_q = off_v + kStages * kv_stage * 2;
-  static constexpr size_t off_p = off_q + kStages * q_slot * 2;                  // float
+  // P of the stage; the merge reuses it as float2 [kDecMaxSplits][G] (same size)
+  static constexpr size_t off_p = off_q + kStages * q_slot * 2;
+  static_assert(kConsumerWarps * kKeysPerWarp * 4 == kDecMaxSplits * 8, "merge scratch");
   static constexpr size_t off_acc = off_p + kConsumerWarps * kKeysPerWarp * G * 4;
   static constexpr size_t off_m = off_acc + size_t(kConsumerWarps) * G * D * 4;
   static constexpr size_t off_l = off_m + kConsumerWarps * G * 4;
   static constexpr size_t off_bar = (off_l + kConsumerWarps * G * 4 + 15) / 16 * 16;
-  static constexpr size_t off_wmax = off_bar + 2 * kStages * 8;  // int per warp
+  static constexpr size_t off_wmax = off_bar + 2 * kStages * 8;  // int per warp, 2 flags
   static constexpr size_t off_prefix = off_wmax + 16 * 4;
-  static size_t bytes(int batch) { return off_prefix + size_t(batch + 1) * 4; }
+  static constexpr size_t off_info(int batch) { return off_prefix + size_t(batch + 1) * 4; }
+  static constexpr size_t bytes(int batch) { return off_info(batch) + size_t(batch) * 4; }
 };
 
-// As many stages (up to 3) as fit in 220 KB of shared memory with a 1024-sequence
-// length table: 3 for every geometry except d = 128 with 8 query heads per KV head.
+// As many stages (up to 3) as fit in the 227 KB of a CTA with 1024-sequence tables:
+// 3 for every geometry except d = 128 with 8 query heads per KV head.
 template <int D, int G>
 using DecodeSmem = DecodeSmemLayout<
-    D, G, (DecodeSmemLayout<D, G, kMaxStages>::off_prefix + 4100 <= 220 * 1024) ? kMaxStages : 2>;
+    D, G, (DecodeSmemLayout<D, G, kMaxStages>::bytes(kDecMaxBatch) <= 227 * 1024) ? kMaxStages : 2>;
 
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeArgs a) {
+template <int D, int G, bool APPEND>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a) {
   using L = DecodeSmem<D, G>;
   constexpr int kStages = L::kStages;
   constexpr int NCH = D / 64;          // 16-byte chunks of a row per lane
@@ -292,27 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
   float* sL = reinterpret_cast<float*>(smem + L::off_l);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   int* prefix = reinterpret_cast<int*>(smem + L::off_prefix);
-  int* wmax = reinterpret_cast<int*>(smem + L::off_wmax);
+  uint32_t* info = reinterpret_cast<uint32_t*>(smem + L::off_info(a.batch));
+  int* wmax = reinterpret_cast<int*>(smem + L::off_wmax);  // [0..8] warp maxima, [13..15] flags
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kStages);
-  pdl_trigger();  // the combine kernel may be scheduled now; it waits for this grid
-  pdl_wait();     // seq_len, the caches and the workspace come from earlier kernels
-
-  // per-sequence stage counts, then an exclusive scan (warp 0) and the largest pair
-  int my_max = 0;
-  for (int b = tid; b < a.batch; b += kThreads) {
-    const Plan p = make_plan(a, b);
-    prefix[b + 1] = a.hkv * p.stages;
-    my_max = max(my_max, p.stages);
-    const int T = a.seq_len[b];
-    if ((T < 0 || T > a.capacity) && blockIdx.x == 0) atomicOr(a.status, kStatusBadLength);
-    if (a.ring_rows > 0 && T > 0 && blockIdx.x == 0 &&
-        route_is_fa(a.fa_mask, a.mask_words, b, a.layer))
-      atomicOr(a.status, kStatusRingRoute);
-  }
-  my_max = __reduce_max_sync(0xffffffffu, my_max);
-  if (lane == 0) wmax[warp] = my_max;
+  const int n_pairs = a.batch * a.hkv;
+  pdl_trigger();  // the next kernel on the stream may be scheduled; it waits for this grid
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -320,7 +379,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
     }
     fence_barrier_init();
   }
+  pdl_wait();  // seq_len, the caches and q may come from earlier kernels
+
+  // Prologue: each sequence's length is read once; keys attended, route, stage counts,
+  // then an exclusive scan (warp 0) and the largest pair.
+  int my_max = 0;
+  for (int b = tid; b < a.batch; b += kThreads) {
+    const int T0 = a.seq_len[b];
+    const bool fa = route_is_fa(a.fa_mask, a.mask_words, b, a.layer);
+    const bool valid = T0 >= 0 && T0 <= a.capacity;
+    const bool ring_fa = a.ring_rows > 0 && fa;  // a ring cache only holds what SA reads
+    int T = 0;
+    if (valid && !ring_fa) {
+      if (!APPEND) {
+        T = T0;
+      } else if (T0 < a.capacity) {
+        T = T0 + 1;
+      } else if (blockIdx.x == 0) {
+        atomicOr(a.status, kStatusCapacity);
+      }
+    }
+    if (blockIdx.x == 0) {
+      if (!valid) atomicOr(a.status, kStatusBadLength);
+      if (ring_fa && (T0 > 0 || APPEND)) atomicOr(a.status, kStatusRingRoute);
+    }
+    info[b] = uint32_t(T) | (fa ? kRouteFa : 0u);
+    const Plan p = make_plan(a, T, fa);
+    prefix[b + 1] = a.hkv * p.stages;
+    my_max = max(my_max, p.stages);
+  }
+  my_max = __reduce_max_sync(0xffffffffu, my_max);
+  if (lane == 0) wmax[warp] = my_max;
   __syncthreads();
+  if (APPEND && tid == kThreads - 1) {
+    // every thread of this CTA has read its lengths; the last CTA to get here advances
+    // them (no CTA of this grid reads seq_len again) and re-zeroes the counter
+    const unsigned old = atomicAdd(a.ws_ctr + kDecCtaCounters - 1, 1u);
+    const bool last = old == gridDim.x - 1;
+    if (last) a.ws_ctr[kDecCtaCounters - 1] = 0u;
+    wmax[14] = last;
+  }
   if (warp == 0) {
     int running = 0;
     for (int base = 0; base < a.batch; base += 32) {
@@ -340,10 +438,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
     if (lane == 0) wmax[15] = m;
   }
   __syncthreads();
+  if (APPEND && wmax[14]) {
+    for (int b = tid; b < a.batch; b += kThreads) {
+      const int T = int(info[b] & ~kRouteFa);
+      if (T > 0) a.seq_len[b] = T;
+    }
+  }
+  // sequences with nothing to attend get zeros, shared out over the grid
+  for (int b = blockIdx.x; b < a.batch; b += gridDim.x) {
+    if ((info[b] & ~kRouteFa) == 0u) {
+      uint16_t* ob = a.o + size_t(b) * a.hkv * G * D;
+      for (int i = tid; i < a.hkv * G * D; i += kThreads) ob[i] = 0;
+    }
+  }
   const int total = prefix[a.batch];
-  const int per = stages_per_cta(total, wmax[15]);
-  const int range0 = min(total, int(blockIdx.x) * per);
-  const int range1 = min(total, range0 + per);
+  int per, range0, range1;
+  if (whole_pairs_pay(total, wmax[15], n_pairs, int(gridDim.x),
+                      float(kStageKeys) * D * 2 * 2)) {
+    // CTA p takes pair p whole: one item, split 0 of 1 (per larger than any range)
+    per = 1 << 30;
+    range0 = range1 = 0;
+    if (int(blockIdx.x) < n_pairs) {
+      const int b = int(blockIdx.x) / a.hkv, kvh = int(blockIdx.x) % a.hkv;
+      const int ns = (prefix[b + 1] - prefix[b]) / a.hkv;
+      range0 = prefix[b] + kvh * ns;
+      range1 = range0 + ns;
+    }
+  } else {
+    per = stages_per_cta(total, wmax[15]);
+    range0 = min(total, int(blockIdx.x) * per);
+    range1 = min(total, range0 + per);
+  }
   const size_t row_elems = D;
 
   if (warp == kConsumerWarps) {
@@ -353,21 +478,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       int g = 0;
       bool ok = true;
       for (int sg = range0; sg < range1 && ok;) {
-        const Item it = item_at(a, prefix, sg, range1, per);
+        const Item it = item_at(a, prefix, info, sg, range1, per);
         sg = it.seg_end;
         const size_t head_off = (size_t(it.b) * a.hkv + it.kvh) * a.rows * row_elems;
-        const uint16_t* qsrc = a.q + (size_t(it.b) * a.hkv * G + size_t(it.kvh) * G) * D;
+        const size_t pair_row = (size_t(it.b) * a.hkv + it.kvh) * D;  // q group / new row
         const int ns = item_stages(it);
         for (int k = 0; k < ns; ++k, ++g) {
-          int row[3], cnt[3], dst[3];
-          const int runs = stage_runs(it, k, row, cnt, dst);
+          int row[3], cnt[3], dst[3], new_dst;
+          const int runs = stage_runs(it, k, APPEND, row, cnt, dst, new_dst);
           const int st = g % kStages;
           const uint32_t ph = (g / kStages) & 1;
           if (!mbar_wait(empty0 + 8 * st, ph ^ 1, a.status)) { ok = false; break; }
           const uint32_t bytes = uint32_t(stage_keys(it, k)) * D * 2;
           const uint32_t qbytes = (k == 0) ? uint32_t(G * D * 2) : 0u;
           mbar_arrive_expect_tx(full0 + 8 * st, 2 * bytes + qbytes);
-          if (k == 0) bulk_g2s(smem_addr(sQ + st * L::q_slot), qsrc, qbytes, full0 + 8 * st, pol);
+          if (k == 0)
+            bulk_g2s(smem_addr(sQ + st * L::q_slot), a.q + pair_row * G, qbytes, full0 + 8 * st, pol);
           for (int r = 0; r < runs; ++r) {
             const uint32_t rb = uint32_t(cnt[r]) * D * 2;
             const size_t src = head_off + size_t(row[r]) * row_elems;
@@ -375,6 +501,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
                      full0 + 8 * st, pol);
             bulk_g2s(smem_addr(sV + st * L::kv_stage + size_t(dst[r]) * D), a.v + src, rb,
                      full0 + 8 * st, pol);
+          }
+          if (APPEND && new_dst >= 0) {
+            bulk_g2s(smem_addr(sK + st * L::kv_stage + size_t(new_dst) * D), a.k_new + pair_row,
+                     D * 2, full0 + 8 * st, pol);
+            bulk_g2s(smem_addr(sV + st * L::kv_stage + size_t(new_dst) * D), a.v_new + pair_row,
+                     D * 2, full0 + 8 * st, pol);
           }
         }
       }
@@ -393,11 +525,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
   const int hl = c >> (3 - GB);            // head this lane holds after group_reduce
   const bool owner = (c & ((1 << (3 - GB)) - 1)) == 0;
   const int group_lane0 = lane & 24;
+  int* flag = wmax + 13;                   // merge flag, shared by the consumer warps
   int g = 0;
   bool ok = true;
-  for (int sg = range0; sg < range1 && ok;) {
-    const Item it = item_at(a, prefix, sg, range1, per);
+  for (int sg = range0; sg < range1;) {
+    const Item it = item_at(a, prefix, info, sg, range1, per);
     sg = it.seg_end;
+    const int pair = it.b * a.hkv + it.kvh;
     uint64_t q2[G][4 * NCH];   // pre-scaled query pairs of this lane's 8*NCH dims
     uint64_t acc[G][4 * NCH];  // P.V pairs of this lane's dims
 #pragma unroll
@@ -406,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       for (int i = 0; i < 4 * NCH; ++i) acc[h][i] = 0ull;
     float m_run = -INFINITY, l_run = 0.f;
 
-    const int ns = item_stages(it);
+    const int ns = ok ? item_stages(it) : 0;
     for (int k = 0; k < ns; ++k, ++g) {
       const int n = stage_keys(it, k);
       const int st = g % kStages;
@@ -513,7 +647,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * st);
     }
-    if (!ok) break;
+    // A piece whose pipeline wait timed out still takes part in its pair's arrival
+    // below (its partial is garbage, the status word says so), so the counters return
+    // to zero as in every call.
 
     // reduce the 4 row groups of the warp, then the 8 warps through shared memory
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
@@ -547,10 +683,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
         sL[warp * G + hl] = l_run;
       }
     }
-    named_barrier_sync(1, kConsumerWarps * 32);
-    const size_t rec = (size_t(it.b) * a.hkv + it.kvh) * kDecMaxSplits + it.split;
-    if (tid == 0 && it.split == 0) a.ws_nsplit[size_t(it.b) * a.hkv + it.kvh] = it.n_split;
-    for (int i = tid; i < G * D; i += kConsumerWarps * 32) {
+    named_barrier_sync(1, kConsumerThreads);
+    uint16_t* out = a.o + size_t(pair) * G * D;
+    const size_t rec0 = size_t(pair) * kDecMaxSplits;
+    for (int i = tid; i < G * D; i += kConsumerThreads) {
       const int h = i / D, e = i % D;
       float M = -INFINITY;
 #pragma unroll
@@ -563,69 +699,85 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const DecodeA
         av = fmaf(f, sAcc[(w * G + h) * D + e], av);
         lv = fmaf(f, sL[w * G + h], lv);
       }
-      a.ws_acc[(rec * G + h) * D + e] = av;
-      if (e == 0) a.ws_ml[rec * G + h] = make_float2(M, lv);
+      if (it.n_split == 1) {
+        const float inv = (lv > 0.f) ? 1.f / lv : 0.f;
+        const __nv_bfloat16 hb = __float2bfloat16_rn(inv * av);
+        out[i] = *reinterpret_cast<const uint16_t*>(&hb);
+      } else {
+        a.ws_acc[(rec0 + it.split) * G * D + i] = av;
+        if (e == 0) a.ws_ml[(rec0 + it.split) * G + h] = make_float2(M, lv);
+      }
     }
-    named_barrier_sync(1, kConsumerWarps * 32);
+    if (APPEND && it.v1 == it.p.n_vis) {
+      // this piece holds the pair's newest key: write its row into the cache
+      const size_t dst = ((size_t(it.b) * a.hkv + it.kvh) * a.rows +
+                          physical_row(a, it.p.n_vis == 0 ? 0 : int(info[it.b] & ~kRouteFa) - 1)) * D;
+      const size_t src = size_t(pair) * D;
+      for (int i = tid; i < 2 * D / 8; i += kConsumerThreads) {
+        const bool is_v = i >= D / 8;
+        const int ch = is_v ? i - D / 8 : i;
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>((is_v ? a.v_new : a.k_new) + src) + ch);
+        // the appending entry points take the caches as writable buffers
+        reinterpret_cast<uint4*>(const_cast<uint16_t*>(is_v ? a.v : a.k) + dst)[ch] = x;
+      }
+    }
+    if (it.n_split > 1) {
+      // publish this piece's partial, then count it; the pair's last piece merges
+      __threadfence();
+      named_barrier_sync(1, kConsumerThreads);
+      if (tid == 0) {
+        const unsigned old = atomicAdd(a.ws_ctr + it.first_cta, 1u);
+        const bool last = old == unsigned(it.n_split - 1);
+        if (last) a.ws_ctr[it.first_cta] = 0u;  // back to zero for the next call
+        *flag = last;
+      }
+      named_barrier_sync(1, kConsumerThreads);
+      if (*flag) {
+        __threadfence();
+        const int nsp = it.n_split;
+        float2* wml = reinterpret_cast<float2*>(sP);  // [kDecMaxSplits][G]: (max, sum)
+        for (int i = tid; i < nsp * G; i += kConsumerThreads) wml[i] = __ldcg(a.ws_ml + rec0 * G + i);
+        named_barrier_sync(1, kConsumerThreads);
+        if (warp < G) {
+          // one warp per query head: splits over the lanes; weights 2^(m_s - M) / L
+          const int h = warp;
+          float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+          if (lane < nsp) { m0 = wml[lane * G + h].x; l0 = wml[lane * G + h].y; }
+          if (lane + 32 < nsp) { m1 = wml[(lane + 32) * G + h].x; l1 = wml[(lane + 32) * G + h].y; }
+          float M = fmaxf(m0, m1);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+          const float f0 = (lane < nsp && m0 != -INFINITY) ? ex2_mufu(m0 - M) : 0.f;
+          const float f1 = (lane + 32 < nsp && m1 != -INFINITY) ? ex2_mufu(m1 - M) : 0.f;
+          float lv = f0 * l0 + f1 * l1;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, off);
+          const float inv = (lv > 0.f) ? 1.f / lv : 0.f;
+          __syncwarp();
+          if (lane < nsp) wml[lane * G + h].x = f0 * inv;
+          if (lane + 32 < nsp) wml[(lane + 32) * G + h].x = f1 * inv;
+        }
+        named_barrier_sync(1, kConsumerThreads);
+        for (int i = tid; i < G * D; i += kConsumerThreads) {
+          const int h = i / D;
+          const float* src = a.ws_acc + rec0 * G * D + i;
+          float av0 = 0.f, av1 = 0.f;
+          int sp = 0;
+          for (; sp + 2 <= nsp; sp += 2) {
+            av0 = fmaf(wml[sp * G + h].x, __ldcg(src + size_t(sp) * G * D), av0);
+            av1 = fmaf(wml[(sp + 1) * G + h].x, __ldcg(src + size_t(sp + 1) * G * D), av1);
+          }
+          if (sp < nsp) av0 = fmaf(wml[sp * G + h].x, __ldcg(src + size_t(sp) * G * D), av0);
+          const __nv_bfloat16 hb = __float2bfloat16_rn(av0 + av1);
+          out[i] = *reinterpret_cast<const uint16_t*>(&hb);
+        }
+      }
+    }
+    named_barrier_sync(1, kConsumerThreads);  // sAcc, sM, sL, sP free for the next item
   }
 }
 
-// Merge the split partials of one (sequence, KV head): weights 2^(m_s - M) / L are
-// computed once per (split, head) in shared memory, then the partial accumulators are
-// read coalesced along d.
-template <int D, int G>
-__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
-  __shared__ float wgt[kDecMaxSplits][G];
-  pdl_trigger();
-  pdl_wait();  // the split kernel's partials
-  const int kvh = blockIdx.x, b = blockIdx.y;
-  const int n_split = make_plan(a, b).n_vis > 0 ? a.ws_nsplit[size_t(b) * a.hkv + kvh] : 0;
-  const size_t rec0 = (size_t(b) * a.hkv + kvh) * kDecMaxSplits;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  if (warp < G) {
-    // one warp per query head of the group: splits spread over the lanes
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    if (lane < n_split) {
-      const float2 ml = a.ws_ml[(rec0 + lane) * G + warp];
-      m0 = ml.x; l0 = ml.y;
-    }
-    if (lane + 32 < n_split) {
-      const float2 ml = a.ws_ml[(rec0 + lane + 32) * G + warp];
-      m1 = ml.x; l1 = ml.y;
-    }
-    float M = fmaxf(m0, m1);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float f0 = (lane < n_split) ? ex2_mufu(m0 - M) : 0.f;
-    const float f1 = (lane + 32 < n_split) ? ex2_mufu(m1 - M) : 0.f;
-    float lv = f0 * l0 + f1 * l1;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) lv += __shfl_xor_sync(0xffffffffu, lv, off);
-    const float inv = (lv > 0.f) ? 1.f / lv : 0.f;
-    if (lane < n_split) wgt[lane][warp] = f0 * inv;
-    if (lane + 32 < n_split) wgt[lane + 32][warp] = f1 * inv;
-  }
-  __syncthreads();
-  uint16_t* out = a.o + (size_t(b) * a.hkv * G + size_t(kvh) * G) * D;
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int gi = i / D, e = i % D;
-    const float* src = a.ws_acc + (rec0 * G + gi) * D + e;
-    float av0 = 0.f, av1 = 0.f, av2 = 0.f, av3 = 0.f;
-    int s = 0;
-    for (; s + 4 <= n_split; s += 4) {
-      av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
-      av1 = fmaf(wgt[s + 1][gi], src[size_t(s + 1) * G * D], av1);
-      av2 = fmaf(wgt[s + 2][gi], src[size_t(s + 2) * G * D], av2);
-      av3 = fmaf(wgt[s + 3][gi], src[size_t(s + 3) * G * D], av3);
-    }
-    for (; s < n_split; ++s) av0 = fmaf(wgt[s][gi], src[size_t(s) * G * D], av0);
-    const __nv_bfloat16 hb = __float2bfloat16_rn((av0 + av1) + (av2 + av3));
-    out[gi * D + e] = *reinterpret_cast<const uint16_t*>(&hb);
-  }
-}
-
-template <int D, int G>
+template <int D, int G, bool APPEND>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   using L = DecodeSmem<D, G>;
   const size_t smem = L::bytes(a.batch);
@@ -641,17 +793,16 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   {
     std::lock_guard<std::mutex> lock(attr_mutex);
     if (!attr_set[dev]) {
-      err = cudaFuncSetAttribute(decode_split_kernel<D, G>,
+      err = cudaFuncSetAttribute(decode_kernel<D, G, APPEND>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(L::bytes(kDecMaxBatch)));
       if (err != cudaSuccess) return err;
       attr_set[dev] = true;
     }
   }
-  err = launch_pdl(decode_split_kernel<D, G>, dim3(device_sm_count()), dim3(kThreads), smem,
-                   stream, a);
-  if (err != cudaSuccess) return err;
-  return launch_pdl(decode_combine_kernel<D, G>, dim3(a.hkv, a.batch), dim3(256), 0, stream, a);
+  const int grid = device_sm_count();
+  if (grid > kDecCtaCounters - 1) return cudaErrorInvalidConfiguration;
+  return launch_pdl(decode_kernel<D, G, APPEND>, dim3(grid), dim3(kThreads), smem, stream, a);
 }
 
 constexpr int kMaxDevices = 64;
@@ -682,13 +833,14 @@ size_t decode_workspace_bytes(const AttnGeom& g, int batch) {
   const int G = g.hq / g.hkv;
   const size_t recs = size_t(batch) * g.hkv * kDecMaxSplits * G;
   const size_t acc = (recs * g.head_dim * 4 + 255) / 256 * 256;
-  return acc + recs * 8 + size_t(batch) * g.hkv * 4;
+  return kDecCounterBytes + acc + recs * 8;
 }
 
 cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
-                          const int32_t* seq_len, int batch, int capacity, int ring_rows,
-                          uint16_t* o, void* workspace, unsigned* status, cudaStream_t stream) {
+                          const uint16_t* k_new, const uint16_t* v_new, int32_t* seq_len,
+                          int batch, int capacity, int ring_rows, uint16_t* o, void* workspace,
+                          unsigned* status, cudaStream_t stream) {
   const int G = g.hq / g.hkv;
   DecodeArgs a;
   a.fa_mask = fa_mask;
@@ -697,6 +849,8 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
   a.q = q;
   a.k = k_cache;
   a.v = v_cache;
+  a.k_new = k_new;
+  a.v_new = v_new;
   a.seq_len = seq_len;
   a.batch = batch;
   a.ring_rows = ring_rows;
@@ -708,14 +862,18 @@ cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
   a.window = g.window;
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(g.head_dim)));
   const size_t recs = size_t(batch) * g.hkv * kDecMaxSplits * G;
-  a.ws_acc = static_cast<float*>(workspace);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.ws_ctr = reinterpret_cast<unsigned*>(ws);
+  a.ws_acc = reinterpret_cast<float*>(ws + kDecCounterBytes);
   const size_t acc_bytes = (recs * g.head_dim * 4 + 255) / 256 * 256;
-  a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + acc_bytes);
-  a.ws_nsplit = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + acc_bytes + recs * 8);
+  a.ws_ml = reinterpret_cast<float2*>(ws + kDecCounterBytes + acc_bytes);
   a.o = o;
   a.status = status;
-#define FLUX_DECODE_CASE(DD, GG) \
-  if (g.head_dim == DD && G == GG) return launch_decode_t<DD, GG>(a, stream);
+  const bool append = k_new != nullptr;
+#define FLUX_DECODE_CASE(DD, GG)                                                   \
+  if (g.head_dim == DD && G == GG)                                                 \
+    return append ? launch_decode_t<DD, GG, true>(a, stream)                       \
+                  : launch_decode_t<DD, GG, false>(a, stream);
   FLUX_DECODE_CASE(128, 1)
   FLUX_DECODE_CASE(128, 2)
   FLUX_DECODE_CASE(128, 4)
@@ -733,13 +891,14 @@ cudaError_t launch_decode_static(const AttnGeom& g, int layer, const uint32_t* f
                                  const uint16_t* v_cache, const int32_t* seq_len, int batch,
                                  int capacity, uint16_t* o, unsigned* status,
                                  cudaStream_t stream) {
-  // The split kernel writes every partial record the combine kernel reads, so the
-  // scratch needs no clearing between calls.
+  // The array starts zeroed and every call leaves its arrival counters at zero; the
+  // partial records need no clearing (each is written before it is read).
   void* scratch = nullptr;
   const cudaError_t err = static_scratch_address(&scratch);
   if (err != cudaSuccess) return err;
-  return launch_decode(g, layer, fa_mask, q, k_cache, v_cache, seq_len, batch, capacity, 0, o,
-                       scratch, status, stream);
+  return launch_decode(g, layer, fa_mask, q, k_cache, v_cache, nullptr, nullptr,
+                       const_cast<int32_t*>(seq_len), batch, capacity, 0, o, scratch, status,
+                       stream);
 }
 
 }  // namespace flux

@@ -236,9 +236,35 @@ int flux_decode(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask
     return FLUX_ERR_WORKSPACE;
   unsigned* status = flux::status_ptr();
   if (!status) return FLUX_ERR_CUDA;
-  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_cache, v_cache, seq_len,
-                                               batch, capacity, 0, o, workspace, status,
+  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_cache, v_cache, nullptr,
+                                               nullptr, const_cast<int32_t*>(seq_len), batch,
+                                               capacity, 0, o, workspace, status,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+int flux_decode_append(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                       const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                       uint16_t* k_cache, uint16_t* v_cache, int32_t* seq_len, int32_t batch,
+                       int32_t capacity, uint16_t* o, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!fa_mask || !q || !k_new || !v_new || !k_cache || !v_cache || !seq_len || !o)
+    return FLUX_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= cfg->n_layers) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > flux::kDecMaxBatch || capacity < 1) return FLUX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) ||
+      !aligned16(v_new))
+    return FLUX_ERR_INVALID_ARG;
+  const flux::AttnGeom g = flux::geom_of(cfg);
+  if (!workspace || workspace_bytes < flux::decode_workspace_bytes(g, batch) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return FLUX_ERR_WORKSPACE;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_cache, v_cache, k_new,
+                                               v_new, seq_len, batch, capacity, 0, o, workspace,
+                                               status, static_cast<cudaStream_t>(stream)));
 }
 
 int flux_decode_static(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
@@ -314,9 +340,36 @@ int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa
     return FLUX_ERR_WORKSPACE;
   unsigned* status = flux::status_ptr();
   if (!status) return FLUX_ERR_CUDA;
-  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_ring, v_ring, seq_len,
-                                               batch, 0, ring_rows, o, workspace, status,
+  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_ring, v_ring, nullptr,
+                                               nullptr, const_cast<int32_t*>(seq_len), batch, 0,
+                                               ring_rows, o, workspace, status,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+int flux_decode_append_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,
+                            const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                            uint16_t* k_ring, uint16_t* v_ring, int32_t* seq_len, int32_t batch,
+                            int32_t ring_rows, uint16_t* o, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  const int st = flux::validate_cfg(cfg);
+  if (st != FLUX_OK) return st;
+  if (!fa_mask || !q || !k_new || !v_new || !k_ring || !v_ring || !seq_len || !o)
+    return FLUX_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= cfg->n_layers) return FLUX_ERR_INVALID_ARG;
+  if (batch < 1 || batch > flux::kDecMaxBatch) return FLUX_ERR_INVALID_ARG;
+  if (ring_rows < cfg->window) return FLUX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(k_new) ||
+      !aligned16(v_new))
+    return FLUX_ERR_INVALID_ARG;
+  const flux::AttnGeom g = flux::geom_of(cfg);
+  if (!workspace || workspace_bytes < flux::decode_workspace_bytes(g, batch) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return FLUX_ERR_WORKSPACE;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  return flux::cuda_status(flux::launch_decode(g, layer, fa_mask, q, k_ring, v_ring, k_new,
+                                               v_new, seq_len, batch, 0, ring_rows, o, workspace,
+                                               status, static_cast<cudaStream_t>(stream)));
 }
 
 int flux_prefill_tile_plan(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,

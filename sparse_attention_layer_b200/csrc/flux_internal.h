@@ -36,15 +36,23 @@ cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
 constexpr int kDecMaxSplits = 64;   // splits per (sequence, KV head)
 constexpr int kDecStageKeys = 128;  // keys per decode pipeline stage
 constexpr int kDecMaxBatch = 1024;
+// Arrival counters at the start of every decode workspace: one per CTA of the grid
+// (a split pair counts its pieces in the counter of the CTA holding its first piece),
+// then one for the appending variant's length update; padded to 256 bytes.
+constexpr int kDecCtaCounters = 1025;
+constexpr size_t kDecCounterBytes = (kDecCtaCounters * 4 + 255) / 256 * 256;
 
 size_t decode_workspace_bytes(const AttnGeom& g, int batch);
 
 // ring_rows == 0: contiguous cache of `capacity` rows per (sequence, KV head);
 // ring_rows > 0: SA ring cache of sink + ring_rows rows (capacity unused).
+// k_new / v_new non-null: the appending variant (one new row per sequence, seq_len
+// advanced); null: seq_len is only read.
 cudaError_t launch_decode(const AttnGeom& g, int layer, const uint32_t* fa_mask,
                           const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
-                          const int32_t* seq_len, int batch, int capacity, int ring_rows,
-                          uint16_t* o, void* workspace, unsigned* status, cudaStream_t stream);
+                          const uint16_t* k_new, const uint16_t* v_new, int32_t* seq_len,
+                          int batch, int capacity, int ring_rows, uint16_t* o, void* workspace,
+                          unsigned* status, cudaStream_t stream);
 
 // Decode with the library's own file-scope scratch array instead of a caller
 // workspace (flux_decode_static).  Its size is FLUX_DECODE_STATIC_SCRATCH_BYTES.

@@ -37,7 +37,8 @@ EXPORTED = (
     "flux_decode_workspace_size", "flux_decode", "flux_sa_block_ranges",
     "flux_get_device_status", "flux_status_string", "flux_version", "flux_decode_static",
     "flux_kv_compact_ring", "flux_kv_append_ring", "flux_decode_ring",
-    "flux_selftest_wait_timeout", "flux_prefill_tile_plan",
+    "flux_selftest_wait_timeout", "flux_prefill_tile_plan", "flux_decode_append",
+    "flux_decode_append_ring",
 )
 
 # flag bit of a flux_prefill_tile_plan entry: the kernel masks keys of that tile
@@ -125,6 +126,12 @@ def lib() -> ctypes.CDLL:
         L.flux_decode.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32, i32,
                                   vp, vp, sz, vp]
         L.flux_decode.restype = ctypes.c_int
+        L.flux_decode_append.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp,
+                                         vp, vp, i32, i32, vp, vp, sz, vp]
+        L.flux_decode_append.restype = ctypes.c_int
+        L.flux_decode_append_ring.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp,
+                                              vp, vp, vp, i32, i32, vp, vp, sz, vp]
+        L.flux_decode_append_ring.restype = ctypes.c_int
         L.flux_decode_static.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, vp, vp, vp, i32,
                                          i32, vp, vp]
         L.flux_decode_static.restype = ctypes.c_int
@@ -275,6 +282,51 @@ def flux_decode(cfg: AttnCfg, layer: int, fa_mask, q, k_cache, v_cache, seq_len,
         _ptr(o, "o", torch.bfloat16, (batch, hq, d)),
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check("flux_decode", st)
+
+
+def flux_decode_append(cfg: AttnCfg, layer: int, fa_mask, q, k_new, v_new, k_cache, v_cache,
+                       seq_len, o, workspace, stream=None) -> None:
+    """One decode step with its KV append in one launch: k_new/v_new [B][1][Hkv][d] go to
+    position seq_len[b], seq_len advances, q [B][Hq][d] attends -> o.  The workspace
+    must have been zero-filled once."""
+    batch, hq, d = q.shape
+    cap = k_cache.shape[2]
+    c = cfg.c()
+    st = lib().flux_decode_append(
+        ctypes.byref(c), int(layer), _ptr(fa_mask, "fa_mask", torch.int32, (batch, cfg.mask_words)),
+        _ptr(q, "q", torch.bfloat16),
+        _ptr(k_new, "k_new", torch.bfloat16, (batch, 1, cfg.n_kv_heads, d)),
+        _ptr(v_new, "v_new", torch.bfloat16, (batch, 1, cfg.n_kv_heads, d)),
+        _ptr(k_cache, "k_cache", torch.bfloat16, (batch, cfg.n_kv_heads, cap, d)),
+        _ptr(v_cache, "v_cache", torch.bfloat16, (batch, cfg.n_kv_heads, cap, d)),
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, cap,
+        _ptr(o, "o", torch.bfloat16, (batch, hq, d)),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("flux_decode_append", st)
+
+
+def flux_decode_append_ring(cfg: AttnCfg, layer: int, fa_mask, q, k_new, v_new, k_ring, v_ring,
+                            seq_len, o, workspace, stream=None) -> None:
+    """flux_decode_append over an SA layer's ring caches [B][Hkv][sink + ring_rows][d]."""
+    batch, hq, d = q.shape
+    rows = k_ring.shape[2]
+    c = cfg.c()
+    st = lib().flux_decode_append_ring(
+        ctypes.byref(c), int(layer), _ptr(fa_mask, "fa_mask", torch.int32, (batch, cfg.mask_words)),
+        _ptr(q, "q", torch.bfloat16),
+        _ptr(k_new, "k_new", torch.bfloat16, (batch, 1, cfg.n_kv_heads, d)),
+        _ptr(v_new, "v_new", torch.bfloat16, (batch, 1, cfg.n_kv_heads, d)),
+        _ptr(k_ring, "k_ring", torch.bfloat16, (batch, cfg.n_kv_heads, rows, d)),
+        _ptr(v_ring, "v_ring", torch.bfloat16, (batch, cfg.n_kv_heads, rows, d)),
+        _ptr(seq_len, "seq_len", torch.int32, (batch,)), batch, rows - cfg.sink,
+        _ptr(o, "o", torch.bfloat16, (batch, hq, d)),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("flux_decode_append_ring", st)
+
+
+def new_decode_workspace(cfg: AttnCfg, batch: int, device="cuda") -> torch.Tensor:
+    """A decode workspace for cfg and batch, zero-filled as the library requires."""
+    return torch.zeros(flux_decode_workspace_size(cfg, batch), dtype=torch.uint8, device=device)
 
 
 def flux_decode_static(cfg: AttnCfg, layer: int, fa_mask, q, k_cache, v_cache, seq_len, o,

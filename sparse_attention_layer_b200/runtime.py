@@ -55,8 +55,7 @@ class HybridAttention:
         n = cfg.n_layers if layers is None else layers
         self.caches = [LayerCache(cfg, batch, capacity, self.device) for _ in range(n)]
         self.fa_mask = torch.zeros(batch, cfg.mask_words, dtype=torch.int32, device=self.device)
-        self.workspace = torch.empty(flux.flux_decode_workspace_size(cfg, batch),
-                                     dtype=torch.uint8, device=self.device)
+        self.workspace = flux.new_decode_workspace(cfg, batch, self.device)
 
     def route(self, w1, b1, w2, b2, xq, pool_len: int = 100, tau: float = 0.0, logits=None):
         flux.flux_route(w1, b1, w2, b2, xq, pool_len, tau, self.fa_mask, logits)
@@ -88,15 +87,14 @@ class HybridAttention:
                 out[:, c0:c1].copy_(oc)
 
     def decode_layer(self, layer: int, q, k_new, v_new, out, cache_index=None):
+        """One decode step of one layer: append the new K/V row and attend, one launch."""
         c = self.caches[layer if cache_index is None else cache_index]
         if isinstance(c, RingCache):
-            flux.flux_kv_append_ring(self.cfg, c.k, c.v, c.seq_len, k_new, v_new)
-            flux.flux_decode_ring(self.cfg, layer, self.fa_mask, q, c.k, c.v, c.seq_len, out,
-                                  self.workspace)
+            flux.flux_decode_append_ring(self.cfg, layer, self.fa_mask, q, k_new, v_new, c.k,
+                                         c.v, c.seq_len, out, self.workspace)
             return
-        flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, k_new, v_new)
-        flux.flux_decode(self.cfg, layer, self.fa_mask, q, c.k, c.v, c.seq_len, out,
-                         self.workspace)
+        flux.flux_decode_append(self.cfg, layer, self.fa_mask, q, k_new, v_new, c.k, c.v,
+                                c.seq_len, out, self.workspace)
 
     def sa_layers(self) -> list:
         """Layers every sequence routes to SA (reads the mask once, after routing:

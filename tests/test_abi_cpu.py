@@ -75,12 +75,12 @@ def _cfg(**kw):
 
 
 def test_workspace_size_formula(L):
-    # per (sequence, KV head, split, query head of the group): d fp32 partials + (max, sum),
-    # then one split count per (sequence, KV head)
+    # 1025 arrival counters padded to 4352 bytes, then per (sequence, KV head, split, query
+    # head of the group): d fp32 partials + (max, sum)
     c = _cfg()
     got = L.flux_decode_workspace_size(ctypes.byref(c), 16)
     recs = 16 * 8 * 64 * 4
-    assert got == (recs * 128 * 4 + 255) // 256 * 256 + recs * 8 + 16 * 8 * 4
+    assert got == 4352 + (recs * 128 * 4 + 255) // 256 * 256 + recs * 8
     bad = _cfg(head_dim=96)
     assert L.flux_decode_workspace_size(ctypes.byref(bad), 16) == 0
     assert L.flux_decode_workspace_size(ctypes.byref(c), 0) == 0
@@ -163,3 +163,17 @@ def test_tile_plan_flag_and_host_checks(L):
                                     None) == flux.FLUX_ERR_INVALID_ARG   # layer out of range
     assert L.flux_prefill_tile_plan(ctypes.byref(c), 0, fake, fake, 1, 1024, 0, fake, 8,
                                     None) == flux.FLUX_OK                # nothing to plan
+
+
+def test_fused_decode_host_checks(L):
+    c = _cfg()
+    fake = ctypes.c_void_p(1 << 20)
+    # missing k_new
+    assert L.flux_decode_append(ctypes.byref(c), 0, fake, fake, None, fake, fake, fake, fake, 1,
+                                1024, fake, fake, 1 << 30, None) == flux.FLUX_ERR_INVALID_ARG
+    # workspace too small
+    assert L.flux_decode_append(ctypes.byref(c), 0, fake, fake, fake, fake, fake, fake, fake, 1,
+                                1024, fake, fake, 16, None) == flux.FLUX_ERR_WORKSPACE
+    # ring shorter than the window
+    assert L.flux_decode_append_ring(ctypes.byref(c), 0, fake, fake, fake, fake, fake, fake, fake,
+                                     1, 1024, fake, fake, 1 << 30, None) == flux.FLUX_ERR_INVALID_ARG

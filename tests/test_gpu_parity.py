@@ -228,7 +228,7 @@ def _decode_case(cfg, ctx, fa_per_seq, steps, seed, capacity=None, layer=0):
     case = CacheCase(cfg, ctx, cap, seed)
     fa_rows = [[layer] if fa else [] for fa in fa_per_seq]
     mask = mask_words(batch, cfg.n_layers, fa_rows).cuda()
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    ws = flux.new_decode_workspace(cfg, batch)
     for step in range(steps):
         kn = inputs.normal_bf16((batch, 1, cfg.n_kv_heads, cfg.head_dim), seed * 31 + step * 3 + 1)
         vn = inputs.normal_bf16((batch, 1, cfg.n_kv_heads, cfg.head_dim), seed * 31 + step * 3 + 2)
@@ -271,7 +271,7 @@ def test_decode_empty_sequence_writes_zeros():
     k = torch.zeros(2, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
     seq = torch.tensor([0, 0], dtype=torch.int32, device="cuda")
     mask = torch.zeros(2, 1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, 2), dtype=torch.uint8, device="cuda")
+    ws = flux.new_decode_workspace(cfg, 2)
     o = torch.full((2, 4, 64), 7.0, dtype=torch.bfloat16, device="cuda")
     q = torch.ones(2, 4, 64, dtype=torch.bfloat16, device="cuda")
     flux.flux_decode(cfg, 0, mask, q, k, k, seq, o, ws)
@@ -284,7 +284,7 @@ def test_decode_bad_length_flag():
     k = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
     seq = torch.tensor([17], dtype=torch.int32, device="cuda")  # past capacity 16
     mask = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, 1), dtype=torch.uint8, device="cuda")
+    ws = flux.new_decode_workspace(cfg, 1)
     o = torch.empty(1, 4, 64, dtype=torch.bfloat16, device="cuda")
     flux.flux_decode(cfg, 0, mask, torch.ones_like(o), k, k, seq, o, ws)
     assert flux.flux_get_device_status() & flux.FLUX_DEVICE_BAD_LENGTH
@@ -420,6 +420,98 @@ def test_decode_pages_sa_geometry(d):
     _decode_case(cfg, ctx, fa, 3, seed=1230 + d, layer=5)
 
 
+@pytest.mark.parametrize("d,group", [(128, 4), (64, 8), (128, 1)])
+def test_decode_append_equals_append_then_decode(d, group):
+    """flux_decode_append (one launch) equals flux_kv_append + flux_decode bit for bit --
+    outputs, cache rows and lengths -- over several steps with ragged lengths, an empty
+    sequence and mixed routes; a sequence without room writes zeros, keeps its rows and
+    length and sets the capacity flag.  The fused outputs also match the oracle."""
+    cfg = AttnCfg(2, 2 * group, 2, d, 64, 64, 256)
+    cap = 2003
+    ctx = [0, 1, 63, 64, 700, 2000, 1999, cap]   # the last one has no room
+    fa = [False, True, False, True, False, False, True, False]
+    batch = len(ctx)
+    sep, fused = CacheCase(cfg, ctx, cap, 77), CacheCase(cfg, ctx, cap, 77)
+    mask = mask_words(batch, cfg.n_layers, [[1] if f else [] for f in fa]).cuda()
+    ws_a, ws_b = flux.new_decode_workspace(cfg, batch), flux.new_decode_workspace(cfg, batch)
+    room = [c < cap for c in ctx]
+    for step in range(3):
+        kn = inputs.normal_bf16((batch, 1, cfg.n_kv_heads, d), 4000 + step).cuda()
+        vn = inputs.normal_bf16((batch, 1, cfg.n_kv_heads, d), 4100 + step).cuda()
+        q = inputs.normal_bf16((batch, cfg.n_q_heads, d), 4200 + step).cuda()
+        o_sep = torch.empty_like(q)
+        o_fused = torch.full_like(q, float("nan"))
+        flux.flux_kv_append(cfg, sep.k, sep.v, sep.seq_len, kn, vn)
+        flux.flux_decode(cfg, 1, mask, q, sep.k, sep.v, sep.seq_len, o_sep, ws_a)
+        assert flux.flux_get_device_status() == flux.FLUX_DEVICE_CAPACITY
+        flux.flux_decode_append(cfg, 1, mask, q, kn, vn, fused.k, fused.v, fused.seq_len, o_fused,
+                                ws_b)
+        torch.cuda.synchronize()
+        assert flux.flux_get_device_status() == flux.FLUX_DEVICE_CAPACITY
+        r = torch.tensor(room)
+        assert torch.equal(o_fused[r], o_sep[r]), f"step {step}"
+        assert (o_fused[~r] == 0).all()
+        assert torch.equal(fused.seq_len, sep.seq_len)
+        assert torch.equal(fused.k.view(torch.int16), sep.k.view(torch.int16))
+        assert torch.equal(fused.v.view(torch.int16), sep.v.view(torch.int16))
+        # mirror the appends on the host copy for the oracle
+        for b in range(batch):
+            if room[b]:
+                t = ctx[b] + step
+                fused.k_host[b, :, t] = kn[b, 0].cpu()
+                fused.v_host[b, :, t] = vn[b, 0].cpu()
+    want = oracle_layer(fused, q.cpu()[:, None], fa)[:, 0]
+    rr = np.array(room)
+    assert_close(f64(o_fused)[rr], want[rr], "fused decode vs oracle")
+    assert (ws_a[:4352] == 0).all() and (ws_b[:4352] == 0).all()  # counters back at zero
+
+
+def test_decode_append_ring_equals_separate_calls():
+    """flux_decode_append_ring equals flux_kv_append_ring + flux_decode_ring bit for bit,
+    and the full-cache fused decode too, across a ring wrap."""
+    cfg = AttnCfg(1, 8, 2, 128, 64, 128, 256)
+    ring_rows = 256
+    ctx = [1, 131, 383, 385, 1000]
+    batch = len(ctx)
+    case_a, k_ra, v_ra, len_a = _ring_setup(cfg, ctx, ring_rows, seed=31)
+    case_b, k_rb, v_rb, len_b = _ring_setup(cfg, ctx, ring_rows, seed=31)
+    mask = mask_words(batch, 1, [[] for _ in ctx]).cuda()
+    ws = [flux.new_decode_workspace(cfg, batch) for _ in range(3)]
+    for step in range(70):   # crosses a block boundary and wraps the ring
+        kn = inputs.normal_bf16((batch, 1, 2, 128), 5000 + step).cuda()
+        vn = inputs.normal_bf16((batch, 1, 2, 128), 5100 + step).cuda()
+        q = inputs.normal_bf16((batch, 8, 128), 5200 + step).cuda()
+        o_sep, o_fused, o_full = (torch.empty_like(q) for _ in range(3))
+        flux.flux_kv_append_ring(cfg, k_ra, v_ra, len_a, kn, vn)
+        flux.flux_decode_ring(cfg, 0, mask, q, k_ra, v_ra, len_a, o_sep, ws[0])
+        flux.flux_decode_append_ring(cfg, 0, mask, q, kn, vn, k_rb, v_rb, len_b, o_fused, ws[1])
+        flux.flux_decode_append(cfg, 0, mask, q, kn, vn, case_b.k, case_b.v, case_b.seq_len,
+                                o_full, ws[2])
+        torch.cuda.synchronize()
+        assert torch.equal(o_fused, o_sep) and torch.equal(o_full, o_sep), f"step {step}"
+        assert torch.equal(len_a, len_b) and torch.equal(k_ra.view(torch.int16), k_rb.view(torch.int16))
+    assert flux.flux_get_device_status() == 0
+
+
+def test_decode_workspace_shared_across_geometries():
+    """One zero-filled workspace serves calls of different batches, routes and split plans
+    in turn (its arrival counters sit at fixed offsets and return to zero)."""
+    cfg = AttnCfg(1, 32, 8, 128, 128, 128, 2048)
+    ws = flux.new_decode_workspace(cfg, 16)
+    for seed, ctx, fa in ((1, [40000], [True]), (2, [3000] * 16, [False] * 16),
+                          (3, [33000] * 4, [True, False, True, True]), (4, [500, 90000], [True, True])):
+        case = CacheCase(cfg, ctx, max(ctx) + 1, 1300 + seed)
+        mask = mask_words(len(ctx), 1, [[0] if f else [] for f in fa]).cuda()
+        q = inputs.normal_bf16((len(ctx), 32, 128), 1400 + seed).cuda()
+        o = torch.empty_like(q)
+        flux.flux_decode(cfg, 0, mask, q, case.k, case.v, case.seq_len, o, ws)
+        torch.cuda.synchronize()
+        assert (ws[:4352] == 0).all(), seed
+        want = oracle_layer(case, q.cpu()[:, None], fa)[:, 0]
+        assert_close(f64(o), want, f"shared workspace call {seed}")
+    assert flux.flux_get_device_status() == 0
+
+
 def test_decode_graph_replay_matches_eager():
     """A decode step captured as a CUDA graph replays to the outputs of the eager calls
     (lengths and routes are read on the device, so the graph serves every step)."""
@@ -511,7 +603,7 @@ def test_ring_decode_identical_to_full(block, sink, window, ring_extra):
     case, k_ring, v_ring, ring_len = _ring_setup(cfg, ctx, ring_rows, seed=9)
     batch = len(ctx)
     mask = mask_words(batch, 1, [[] for _ in ctx]).cuda()
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    ws = flux.new_decode_workspace(cfg, batch)
     for step in range(block + 3):   # crosses a block boundary and wraps the ring
         kn = inputs.normal_bf16((batch, 1, 2, 128), 500 + step)
         vn = inputs.normal_bf16((batch, 1, 2, 128), 600 + step)
@@ -535,7 +627,7 @@ def test_ring_decode_refuses_fa_route():
     k = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
     seq = torch.tensor([100], dtype=torch.int32, device="cuda")
     mask = torch.ones(1, 1, dtype=torch.int32, device="cuda")  # layer 0 routed to FA
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, 1), dtype=torch.uint8, device="cuda")
+    ws = flux.new_decode_workspace(cfg, 1)
     o = torch.full((1, 4, 64), 3.0, dtype=torch.bfloat16, device="cuda")
     flux.flux_decode_ring(cfg, 0, mask, torch.ones_like(o), k, k, seq, o, ws)
     assert flux.flux_get_device_status() & flux.FLUX_DEVICE_RING_ROUTE
@@ -550,8 +642,7 @@ def test_ring_decode_llama_full_size():
     ctx = [w.seq] * w.batch
     case, k_ring, v_ring, ring_len = _ring_setup(cfg, ctx, w.window, seed=1002)
     mask = mask_words(w.batch, cfg.n_layers, [[] for _ in ctx]).cuda()
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, w.batch), dtype=torch.uint8,
-                     device="cuda")
+    ws = flux.new_decode_workspace(cfg, w.batch)
     for step in range(2):
         kn = inputs.normal_bf16((w.batch, 1, 8, 128), 800 + step)
         vn = inputs.normal_bf16((w.batch, 1, 8, 128), 900 + step)

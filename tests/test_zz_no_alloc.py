@@ -38,7 +38,7 @@ def test_static_scratch_decode_matches_workspace_decode():
     batch = len(ctx)
     case = CacheCase(cfg, ctx, 6000, seed=4242)
     mask = mask_words(batch, cfg.n_layers, [[0], [], [0, 1], []]).cuda()
-    ws = torch.empty(flux.flux_decode_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    ws = flux.new_decode_workspace(cfg, batch)
     qs = [inputs.normal_bf16((batch, cfg.n_q_heads, cfg.head_dim), 9000 + call).cuda()
           for call in range(2)]
     o_ws = [torch.empty_like(q) for q in qs]
