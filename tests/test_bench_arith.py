@@ -62,3 +62,13 @@ def test_llama_decode_and_prefill_figures(bench):
     assert sa == 2 * 2 * 16 * 8 * 128 * (128 + 1 + 15 * 128) + 2 * 2 * 16 * 32 * 128
     # causal FA over 8192 tokens: sum of (t + 1) visible keys per query row
     assert bench.prefill_flops_per_layer(c, 8192, True) == 4.0 * 128 * 32 * 8192 * 8193 / 2
+
+
+def test_fused_append_adds_the_new_rows(bench):
+    """A flux_decode_append launch also writes one K and one V row per (sequence, KV head)."""
+    c = cfg()
+    w = SimpleNamespace(batch=16)
+    for fa in (True, False):
+        plain = bench.decode_bytes_per_layer(w, c, 32769, fa)
+        fused = bench.decode_bytes_per_layer(w, c, 32769, fa, append=True)
+        assert fused - plain == 2 * 2 * 16 * 8 * 128
