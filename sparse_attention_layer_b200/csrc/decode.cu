@@ -59,8 +59,21 @@ namespace {
 constexpr int kStageKeys = kDecStageKeys;
 constexpr int kMaxStages = 3;
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+// Three warpgroups: two of consumers (warps 0-7) and one whose first lane is the
+// producer.  A block of 384 threads launches with 168 registers per thread (three
+// warps per SM sub-partition); the producer warpgroup then gives most of its registers
+// back (setmaxnreg.dec to kProducerRegs) and the consumers take them
+// (setmaxnreg.inc to kConsumerRegs): 256 x 232 + 128 x 40 = 64512 = 384 x 168, the
+// registers the block was launched with, so the increase never waits.  With 168 the
+// consumers spilled.
+constexpr int kThreads = 384;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 40;
+constexpr int kConsumerRegs = 232;
+static_assert(kConsumerThreads * kConsumerRegs + (kThreads - kConsumerThreads) * kProducerRegs <=
+                  kThreads * kLaunchRegs,
+              "register split above the launch allocation");
 constexpr int kKeysPerWarp = kStageKeys / kConsumerWarps;  // 16 keys per warp per stage
 constexpr int kPasses = kKeysPerWarp / 4;                  // 4 keys per warp instruction
 static_assert(kPasses == 4, "the tile maximum below is written for 4 passes");
@@ -471,9 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   }
   const size_t row_elems = D;
 
-  if (warp == kConsumerWarps) {
+  if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == kConsumerWarps && lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
       int g = 0;
       bool ok = true;
@@ -520,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   }
 
   // ------------------------------------------------------------------ consumers
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
   const int key_sub = lane >> 3;           // which of the 4 rows of a warp instruction
   const int c = lane & 7;                  // 16-byte chunk within the row
   const int hl = c >> (3 - GB);            // head this lane holds after group_reduce
@@ -567,9 +582,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 #pragma unroll
       for (int p = 0; p < kPasses; ++p) {
         const int key = warp * kKeysPerWarp + p * 4 + key_sub;
-        uint64_t dot2[G];
+        // two accumulation chains per head (even / odd words) halve the dependent FMAs
+        uint64_t dot2[G], dot2b[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) dot2[h] = 0ull;
+        for (int h = 0; h < G; ++h) dot2[h] = dot2b[h] = 0ull;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
           const uint4 raw = lds128(Ks + key * D + ch * 64 + c * 8);
@@ -578,16 +594,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             dot2[h] = f2_fma(q2[h][ch * 4 + 0], k0, dot2[h]);
-            dot2[h] = f2_fma(q2[h][ch * 4 + 1], k1, dot2[h]);
+            dot2b[h] = f2_fma(q2[h][ch * 4 + 1], k1, dot2b[h]);
             dot2[h] = f2_fma(q2[h][ch * 4 + 2], k2, dot2[h]);
-            dot2[h] = f2_fma(q2[h][ch * 4 + 3], k3, dot2[h]);
+            dot2b[h] = f2_fma(q2[h][ch * 4 + 3], k3, dot2b[h]);
           }
         }
         float dot[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float lo, hi;
-          f2_unpack(dot2[h], lo, hi);
+          f2_unpack(f2_add(dot2[h], dot2b[h]), lo, hi);
           dot[h] = lo + hi;
         }
         const float r = group_reduce<G>(dot, lane);
