@@ -6,7 +6,9 @@
 prefill: one Llama-3.1-8B-shaped layer, 8192-token prompt (Q 64 MB, K/V 16 MB each,
          O 64 MB: more than the 126 MB L2 together), FA route unless --sa.
 decode:  one Llama-shaped layer, `batch` sequences at 32768 context (K+V 134 MB per
-         sequence), FA route unless --sa.
+         sequence), FA route unless --sa; each launch is the decode step's
+         flux_decode_append (the new row is appended, so launch i attends 32769 + i keys,
+         as the bench's decode steps do).
 Each launch is timed with CUDA events; the script prints one JSON line.
 """
 
@@ -57,18 +59,20 @@ def main():
     else:
         T = args.seq or 32768
         B = args.batch
-        m = HybridAttention(cfg, B, T + 1, "cuda")
+        m = HybridAttention(cfg, B, T + args.launches, "cuda")
         m.set_mask(inputs.pack_bits_u32(bits).cuda())
         c = m.caches[0]
         c.k.normal_(generator=gen)
         c.v.normal_(generator=gen)
         c.seq_len.fill_(T)
         q = torch.randn(B, 32, 128, device="cuda", generator=gen).to(torch.bfloat16)
+        kn = torch.randn(B, 1, 8, 128, device="cuda", generator=gen).to(torch.bfloat16)
         o = torch.empty_like(q)
         for _ in range(args.launches):
             a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
             a.record()
-            flux.flux_decode(cfg, 0, m.fa_mask, q, c.k, c.v, c.seq_len, o, m.workspace)
+            flux.flux_decode_append(cfg, 0, m.fa_mask, q, kn, kn, c.k, c.v, c.seq_len, o,
+                                    m.workspace)
             b.record()
             times.append((a, b))
         n_units = B
