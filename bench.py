@@ -748,6 +748,42 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
         v["speedup_vs_all_fa"] = base / v["ms_per_step"]
     clocks = sampler.stop()
     pb.fa = pb.mask_bits(pb.router_mask)
+    pb.model.set_mask(pb.router_mask)
+
+    # end to end from pinned host buffers: per step x_Q in for the router, then per layer
+    # q, k, v in and o out (layer inputs arrive and outputs leave as the layers run)
+    from sparse_attention_layer_b200 import flux
+    xq_h = pb.xq.cpu().pin_memory()
+    q_h, k_h, v_h = (t.cpu().pin_memory() for t in (pb.q, pb.k, pb.v))
+    o_h = torch.empty(pb.o.shape, dtype=pb.o.dtype).pin_memory()
+    m = pb.model
+    e2e_steps = 3
+    barrier(world)
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(e2e_steps):
+        pb.reset()
+        pb.xq.copy_(xq_h, non_blocking=True)
+        m.route(*pb.router, pb.xq, w.pool_len, w.tau)
+        for layer in range(w.n_layers):
+            pb.q.copy_(q_h, non_blocking=True)
+            pb.k.copy_(k_h, non_blocking=True)
+            pb.v.copy_(v_h, non_blocking=True)
+            c = m.caches[layer]
+            flux.flux_kv_append(pb.cfg, c.k, c.v, c.seq_len, pb.k, pb.v)
+            flux.flux_prefill(pb.cfg, layer, m.fa_mask, pb.q, c.k, c.v, c.seq_len, pb.o)
+            o_h.copy_(pb.o, non_blocking=True)
+    e2.record()
+    barrier(world)
+    t_e2e = max_over_ranks(s2.elapsed_time(e2), world) / e2e_steps
+    e2e = {"value": world * w.batch * w.seq / (t_e2e / 1e3), "unit": "tokens/s",
+           "ms_per_step": t_e2e,
+           "h2d_bytes_per_step": xq_h.numel() * 2 + w.n_layers * (q_h.numel() + k_h.numel() +
+                                                                 v_h.numel()) * 2,
+           "d2h_bytes_per_step": w.n_layers * o_h.numel() * 2,
+           "what": "per step: pinned-host x_Q copied in and routed, then per layer pinned-host "
+                   "q, k, v copied in, KV append + prefill, the layer's output copied out"}
     out = {
         "workload": "llama3.1-8b-shape prefill, 1 x 8192 tokens, router 4096->256->32 "
                     f"(seeded; {w.n_layers - n_fa} SA layers), SA sink 128 + window 2048",
@@ -762,11 +798,12 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
                                        statistics.mean(elapsed_ms(sa_ev)), peaks, peak_kind,
                                        clocks),
         "routing_mix": mix,
+        "e2e": e2e,
         "gpu_launches_per_step": pb.launches_per_step,
         "clocks": clocks,
         "cpu_baseline": None,
     }
-    del pb
+    del pb, xq_h, q_h, k_h, v_h, o_h
     torch.cuda.empty_cache()
     if world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_prefill_baseline(w, n_fa)

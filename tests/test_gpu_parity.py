@@ -512,6 +512,35 @@ def test_decode_workspace_shared_across_geometries():
     assert flux.flux_get_device_status() == 0
 
 
+def test_decode_append_batch_limit():
+    """1024 sequences (the decode batch limit: the per-sequence length table and stage
+    prefix fill the kernel's shared-memory tables), ragged lengths from 0 to 600, mixed
+    routes, the fused append; outputs against the oracle and lengths advanced by one."""
+    cfg = AttnCfg(2, 8, 2, 64, 64, 64, 256)
+    batch = 1024
+    ctx = inputs.random_seq_lens(batch, 0, 600, seed=31).tolist()
+    cap = 608
+    case = CacheCase(cfg, ctx, cap, seed=1240)
+    fa = [(b * 7) % 3 == 0 for b in range(batch)]
+    mask = mask_words(batch, cfg.n_layers, [[1] if f else [] for f in fa]).cuda()
+    ws = flux.new_decode_workspace(cfg, batch)
+    kn = inputs.normal_bf16((batch, 1, 2, 64), 1241)
+    vn = inputs.normal_bf16((batch, 1, 2, 64), 1242)
+    q = inputs.normal_bf16((batch, 8, 64), 1243)
+    o = torch.empty(batch, 8, 64, dtype=torch.bfloat16, device="cuda")
+    flux.flux_decode_append(cfg, 1, mask, q.cuda(), kn.cuda(), vn.cuda(), case.k, case.v,
+                            case.seq_len, o, ws)
+    torch.cuda.synchronize()
+    assert flux.flux_get_device_status() == 0
+    assert case.seq_len.cpu().tolist() == [c + 1 for c in ctx]
+    for b in range(batch):
+        case.k_host[b, :, ctx[b]] = kn[b, 0]
+        case.v_host[b, :, ctx[b]] = vn[b, 0]
+    want = oracle_layer(case, q[:, None], fa)[:, 0]
+    assert_close(f64(o), want, "decode at batch 1024")
+    assert (ws[:4352] == 0).all()
+
+
 def test_decode_graph_replay_matches_eager():
     """A decode step captured as a CUDA graph replays to the outputs of the eager calls
     (lengths and routes are read on the device, so the graph serves every step)."""
