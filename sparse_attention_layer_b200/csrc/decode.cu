@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   int* prefix = reinterpret_cast<int*>(smem + L::off_prefix);
   uint32_t* info = reinterpret_cast<uint32_t*>(smem + L::off_info(a.batch));
-  int* wmax = reinterpret_cast<int*>(smem + L::off_wmax);  // [0..8] warp maxima, [13..15] flags
+  int* wmax = reinterpret_cast<int*>(smem + L::off_wmax);  // [0..11] warp maxima, [13, 15] flags
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kStages);
@@ -424,14 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   my_max = __reduce_max_sync(0xffffffffu, my_max);
   if (lane == 0) wmax[warp] = my_max;
   __syncthreads();
-  if (APPEND && tid == kThreads - 1) {
-    // every thread of this CTA has read its lengths; the last CTA to get here advances
-    // them (no CTA of this grid reads seq_len again) and re-zeroes the counter
-    const unsigned old = atomicAdd(a.ws_ctr + kDecCtaCounters - 1, 1u);
-    const bool last = old == gridDim.x - 1;
-    if (last) a.ws_ctr[kDecCtaCounters - 1] = 0u;
-    wmax[14] = last;
-  }
   if (warp == 0) {
     int running = 0;
     for (int base = 0; base < a.batch; base += 32) {
@@ -451,12 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     if (lane == 0) wmax[15] = m;
   }
   __syncthreads();
-  if (APPEND && wmax[14]) {
-    for (int b = tid; b < a.batch; b += kThreads) {
-      const int T = int(info[b] & ~kRouteFa);
-      if (T > 0) a.seq_len[b] = T;
-    }
-  }
   // sequences with nothing to attend get zeros, shared out over the grid
   for (int b = blockIdx.x; b < a.batch; b += gridDim.x) {
     if ((info[b] & ~kRouteFa) == 0u) {
@@ -487,6 +473,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (APPEND && warp == kConsumerWarps + 1) {
+      // Off the consumers' path: every thread of this CTA has read its lengths (before
+      // the first barrier); the last CTA to arrive advances them (no CTA of this grid
+      // reads seq_len again) and re-zeroes the counter.
+      unsigned last = 0u;
+      if (lane == 0) {
+        last = atomicAdd(a.ws_ctr + kDecCtaCounters - 1, 1u) == gridDim.x - 1;
+        if (last) a.ws_ctr[kDecCtaCounters - 1] = 0u;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        for (int b = lane; b < a.batch; b += 32) {
+          const int T = int(info[b] & ~kRouteFa);
+          if (T > 0) a.seq_len[b] = T;
+        }
+      }
+    }
     if (warp == kConsumerWarps && lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
       int g = 0;
