@@ -460,13 +460,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // memory, so the S buffer is free before P_j V_j runs -- and P_j V_j as soon as P_j
       // (p_full) and V_j have landed.  Polling uses the non-blocking test.
       int s_next[2] = {2, 3}, pv_next[2] = {0, 1};
-      unsigned long long t_last = global_ns();
+      // The clock is read only after 256 idle polls in a row, never on a productive
+      // pass: the loop's latency is the MMAs' reaction time.  A wait is thus bounded by
+      // the limit plus 256 polls.
+      unsigned idle = 0;
+      unsigned long long t_idle = 0;
       while (ok && (pv_next[0] < n || pv_next[1] < n)) {
         bool progress = false;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           const int js = s_next[g];
-          if (js < n && mbar_test(bar_sfree + 8 * g, ((js - 2) >> 1) & 1) &&
+          // K_js refills the slot of K_{js-KS}.  A parity test on the slot is exact only
+          // once that earlier fill is known to have landed, i.e. once S_{js-KS} has been
+          // issued (with KS = 3 it belongs to the other warpgroup); K_js cannot land
+          // before that anyway, since S_{js-KS} has to release the slot first.  The
+          // index (g + KS) & 1 is a constant of the unrolled loop (a dynamic one would put
+          // s_next in local memory, on this thread's critical path).
+          const int t_prev = js - KS;
+          const bool prev_seen = (KS % 2 == 0) || t_prev < 0 || s_next[(g + KS) & 1] > t_prev;
+          if (js < n && prev_seen && mbar_test(bar_sfree + 8 * g, ((js - 2) >> 1) & 1) &&
               mbar_test(bar_kfull + 8 * (js % KS), (js / KS) & 1)) {
             issue_s(js);
             s_next[g] = js + 2;
@@ -474,6 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int j = pv_next[g];
           if (j >= n) continue;
+          // V_j refills the slot of V_{j-2}, read by P_{j-2} V_{j-2} of this warpgroup,
+          // already issued: the parity test is exact
+          static_assert(kVStages == 2, "V slot reuse must stay within one warpgroup");
           const int st = j % kVStages;
           if (!mbar_test(bar_pfull + 8 * g, (j >> 1) & 1)) continue;
           if (!mbar_test(bar_vfull + 8 * st, (j / kVStages) & 1)) continue;
@@ -492,10 +507,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           progress = true;
         }
         if (progress) {
-          t_last = global_ns();
-        } else if (global_ns() - t_last > kWaitLimitNs) {
-          atomicOr(a.status, kStatusTimeout);
-          ok = false;
+          idle = 0;
+        } else if ((++idle & 255u) == 0u) {
+          const unsigned long long now = global_ns();
+          if (idle == 256u) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitLimitNs) {
+            atomicOr(a.status, kStatusTimeout);
+            ok = false;
+          }
         }
       }
       // every MMA this thread issued has finished before tensor memory is freed
