@@ -67,6 +67,9 @@ typedef enum flux_status {
 #define FLUX_DEVICE_RING_ROUTE 0x8u /* flux_decode_ring saw a sequence routed to FA */
 #define FLUX_DEVICE_LAYOUT 0x10u    /* prefill: dynamic shared memory not 1024-byte aligned;
                                        nothing computed (never seen on B200) */
+#define FLUX_DEVICE_BOUNDS 0x20u    /* checked build only: a guarded global access (decode
+                                       copies, cache and workspace writes, KV appends)
+                                       would have left its buffer; it was skipped */
 
 /* Attention geometry of one model; the same struct serves every layer. */
 typedef struct flux_attn_cfg {
@@ -310,6 +313,21 @@ int flux_prefill_tile_plan(const flux_attn_cfg* cfg, int32_t layer, const uint32
  * microseconds (1..1000000).  The wait gives up, FLUX_DEVICE_TIMEOUT is set in the
  * device status word and the kernel returns; the context stays usable. */
 int flux_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/* Checked build (libflux_checked.so: every kernel compiled with FLUX_CHECKED): global
+ * accesses whose indices come from run-time data -- the decode kernel's K/V/q copies,
+ * its cache-row and split-partial writes and arrival counters, every KV append and
+ * ring compaction -- are guarded; a failing guard sets FLUX_DEVICE_BOUNDS and skips the
+ * access, nothing traps.  (Prefill reads K/V only through TMA boxes, which the hardware
+ * bounds, and writes rows < n_q by construction.)  The plain libflux.so compiles the
+ * guards away.  Same exported symbols, same results.
+ *
+ * flux_build_checked -- 1 in the checked build, 0 in the plain one (host only).
+ * flux_selftest_bounds -- a guard refuses index 16 of a 16-entry device array: the
+ *   checked build sets FLUX_DEVICE_BOUNDS, the plain build leaves the status word as it
+ *   was; neither touches memory outside the array. */
+int flux_build_checked(void);
+int flux_selftest_bounds(void* stream);
 
 /* Copy the device status word of the current device to *bits and clear it.
  * Synchronises `stream` first. */

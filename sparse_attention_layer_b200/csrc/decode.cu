@@ -509,17 +509,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           const uint32_t bytes = uint32_t(stage_keys(it, k)) * D * 2;
           const uint32_t qbytes = (k == 0) ? uint32_t(G * D * 2) : 0u;
           mbar_arrive_expect_tx(full0 + 8 * st, 2 * bytes + qbytes);
-          if (k == 0)
+          if (k == 0 && FLUX_IN_BOUNDS(it.b < a.batch && it.kvh < a.hkv, a.status))
             bulk_g2s(smem_addr(sQ + st * L::q_slot), a.q + pair_row * G, qbytes, full0 + 8 * st, pol);
           for (int r = 0; r < runs; ++r) {
             const uint32_t rb = uint32_t(cnt[r]) * D * 2;
             const size_t src = head_off + size_t(row[r]) * row_elems;
+            // (a skipped copy leaves its stage short: the consumers' wait then times out)
+            if (!FLUX_IN_BOUNDS(row[r] >= 0 && row[r] + cnt[r] <= a.rows && dst[r] >= 0 &&
+                                    dst[r] + cnt[r] <= kStageKeys,
+                                a.status))
+              continue;
             bulk_g2s(smem_addr(sK + st * L::kv_stage + size_t(dst[r]) * D), a.k + src, rb,
                      full0 + 8 * st, pol);
             bulk_g2s(smem_addr(sV + st * L::kv_stage + size_t(dst[r]) * D), a.v + src, rb,
                      full0 + 8 * st, pol);
           }
-          if (APPEND && new_dst >= 0) {
+          if (APPEND && new_dst >= 0 && FLUX_IN_BOUNDS(new_dst < kStageKeys, a.status)) {
             bulk_g2s(smem_addr(sK + st * L::kv_stage + size_t(new_dst) * D), a.k_new + pair_row,
                      D * 2, full0 + 8 * st, pol);
             bulk_g2s(smem_addr(sV + st * L::kv_stage + size_t(new_dst) * D), a.v_new + pair_row,
@@ -723,14 +728,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         const __nv_bfloat16 hb = __float2bfloat16_rn(inv * av);
         out[i] = *reinterpret_cast<const uint16_t*>(&hb);
       } else {
-        a.ws_acc[(rec0 + it.split) * G * D + i] = av;
-        if (e == 0) a.ws_ml[(rec0 + it.split) * G + h] = make_float2(M, lv);
+        if (FLUX_IN_BOUNDS(it.split < kDecMaxSplits, a.status)) {
+          a.ws_acc[(rec0 + it.split) * G * D + i] = av;
+          if (e == 0) a.ws_ml[(rec0 + it.split) * G + h] = make_float2(M, lv);
+        }
       }
     }
-    if (APPEND && it.v1 == it.p.n_vis) {
+    const int new_row = physical_row(a, it.p.n_vis == 0 ? 0 : int(info[it.b] & ~kRouteFa) - 1);
+    if (APPEND && it.v1 == it.p.n_vis &&
+        FLUX_IN_BOUNDS(new_row >= 0 && new_row < a.rows, a.status)) {
       // this piece holds the pair's newest key: write its row into the cache
-      const size_t dst = ((size_t(it.b) * a.hkv + it.kvh) * a.rows +
-                          physical_row(a, it.p.n_vis == 0 ? 0 : int(info[it.b] & ~kRouteFa) - 1)) * D;
+      const size_t dst = ((size_t(it.b) * a.hkv + it.kvh) * a.rows + new_row) * D;
       const size_t src = size_t(pair) * D;
       for (int i = tid; i < 2 * D / 8; i += kConsumerThreads) {
         const bool is_v = i >= D / 8;
@@ -740,7 +748,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         reinterpret_cast<uint4*>(const_cast<uint16_t*>(is_v ? a.v : a.k) + dst)[ch] = x;
       }
     }
-    if (it.n_split > 1) {
+    if (it.n_split > 1 && FLUX_IN_BOUNDS(it.first_cta < kDecCtaCounters - 1 &&
+                                             it.n_split <= kDecMaxSplits,
+                                         a.status)) {
       // publish this piece's partial, then count it; the pair's last piece merges
       __threadfence();
       named_barrier_sync(1, kConsumerThreads);

@@ -63,6 +63,16 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned* stat
   mbar_wait(b, 0, status, limit_ns);
 }
 
+// Bounds-guard self-test: a guard refuses index 16 of a 16-entry array.  The checked
+// build records FLUX_DEVICE_BOUNDS; the plain build compiles the guard to true, and the
+// index check that follows it keeps the access out either way.
+__device__ unsigned g_bounds_probe[16];
+
+__global__ void selftest_bounds_kernel(int index, unsigned* status) {
+  const bool inside = index >= 0 && index < 16;
+  if (FLUX_IN_BOUNDS(inside, status) && inside) g_bounds_probe[index] = 1u;
+}
+
 int validate_cfg(const flux_attn_cfg* c) {
   if (!c) return FLUX_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->n_layers > 1024) return FLUX_ERR_INVALID_ARG;
@@ -146,6 +156,21 @@ int flux_selftest_wait_timeout(uint32_t limit_us, void* stream) {
   flux::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       (unsigned long long)limit_us * 1000ull, status);
   return flux::cuda_status(cudaGetLastError());
+}
+
+int flux_selftest_bounds(void* stream) {
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
+  flux::selftest_bounds_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(16, status);
+  return flux::cuda_status(cudaGetLastError());
+}
+
+int flux_build_checked(void) {
+#ifdef FLUX_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 int flux_get_device_status(void* stream, uint32_t* bits) {
@@ -318,9 +343,12 @@ int flux_kv_append_ring(const flux_attn_cfg* cfg, uint16_t* k_ring, uint16_t* v_
   if (!aligned16(k_ring) || !aligned16(v_ring) || !aligned16(k_new) || !aligned16(v_new))
     return FLUX_ERR_INVALID_ARG;
   if (n_new == 0) return FLUX_OK;
+  unsigned* status = flux::status_ptr();
+  if (!status) return FLUX_ERR_CUDA;
   return flux::cuda_status(flux::launch_kv_append_ring(flux::geom_of(cfg), k_ring, v_ring,
                                                        seq_len, batch, ring_rows, k_new, v_new,
-                                                       n_new, static_cast<cudaStream_t>(stream)));
+                                                       n_new, status,
+                                                       static_cast<cudaStream_t>(stream)));
 }
 
 int flux_decode_ring(const flux_attn_cfg* cfg, int32_t layer, const uint32_t* fa_mask,

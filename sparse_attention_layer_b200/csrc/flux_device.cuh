@@ -22,6 +22,18 @@ constexpr unsigned kStatusTimeout = 0x2u;
 constexpr unsigned kStatusBadLength = 0x4u;
 constexpr unsigned kStatusRingRoute = 0x8u;
 constexpr unsigned kStatusLayout = 0x10u;
+constexpr unsigned kStatusBounds = 0x20u;
+
+// Bounds guards of the checked build (compiled with FLUX_CHECKED: libflux_checked.so).
+// A guard whose condition fails records kStatusBounds in the status word and the access
+// it guards is skipped; nothing traps.  In the plain build FLUX_IN_BOUNDS(...) is the
+// constant true, the condition is not even evaluated, and the access runs as the
+// host-side argument checks and the kernel's own logic allow.
+#ifdef FLUX_CHECKED
+#define FLUX_IN_BOUNDS(cond, status) ::flux::bounds_ok((cond), (status))
+#else
+#define FLUX_IN_BOUNDS(cond, status) true
+#endif
 
 // A pipeline wait gives up after this long (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -100,6 +112,11 @@ __device__ __forceinline__ bool route_is_fa(const uint32_t* fa_mask, int mask_wo
 }
 
 // ------------------------------------------------------------------ small utilities
+
+__device__ __forceinline__ bool bounds_ok(bool cond, unsigned* status) {
+  if (!cond) atomicOr(status, kStatusBounds);
+  return cond;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -76,7 +76,7 @@ cudaError_t launch_kv_compact_ring(const AttnGeom& g, const uint16_t* k_cache,
 cudaError_t launch_kv_append_ring(const AttnGeom& g, uint16_t* k_ring, uint16_t* v_ring,
                                   int32_t* seq_len, int batch, int ring_rows,
                                   const uint16_t* k_new, const uint16_t* v_new, int n_new,
-                                  cudaStream_t stream);
+                                  unsigned* status, cudaStream_t stream);
 
 // ----- router
 constexpr int kRouterMaxHidden = 16384;

@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(256) kv_append_copy_kernel(
     const long long rest = i / chunks_per_row;
     const int kvh = int(rest % hkv);
     const int tok = int(rest / hkv);
+    if (!FLUX_IN_BOUNDS(start + tok < capacity, status)) continue;
     const size_t dst = ((size_t(b) * hkv + kvh) * capacity + start + tok) * row_elems + ch * 8;
     const uint4 kv = __ldg(ks + i);
     const uint4 vv = __ldg(vs + i);
@@ -73,6 +74,7 @@ __global__ void __launch_bounds__(256) kv_append_fused_kernel(
       const int rest = i / chunks_per_row;
       const int kvh = rest % hkv;
       const int tok = rest / hkv;
+      if (!FLUX_IN_BOUNDS(start + tok < capacity, status)) continue;
       const size_t dst = ((size_t(b) * hkv + kvh) * capacity + start + tok) * row_elems + ch * 8;
       *reinterpret_cast<uint4*>(k_cache + dst) = __ldg(ks + i);
       *reinterpret_cast<uint4*>(v_cache + dst) = __ldg(vs + i);
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(256) kv_append_ring_kernel(
     uint16_t* __restrict__ k_ring, uint16_t* __restrict__ v_ring,
     const int32_t* __restrict__ seq_len, int sink, int ring_rows,
     const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new, int n_new, int hkv,
-    int chunks_per_row) {
+    int chunks_per_row, unsigned* status) {
   const int b = blockIdx.y;
   const int start = seq_len[b];
   if (start < 0) return;
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(256) kv_append_ring_kernel(
     const int kvh = int(rest % hkv);
     const int tok = int(rest / hkv);
     const int slot = ring_slot(start + tok, sink, ring_rows);
+    if (!FLUX_IN_BOUNDS(slot >= 0 && slot < rows, status)) continue;
     const size_t dst = ((size_t(b) * hkv + kvh) * rows + slot) * row_elems + ch * 8;
     *reinterpret_cast<uint4*>(k_ring + dst) = __ldg(ks + i);
     *reinterpret_cast<uint4*>(v_ring + dst) = __ldg(vs + i);
@@ -128,7 +131,7 @@ __global__ void __launch_bounds__(256) kv_append_ring_kernel(
 __global__ void __launch_bounds__(256) kv_append_ring_fused_kernel(
     uint16_t* __restrict__ k_ring, uint16_t* __restrict__ v_ring, int32_t* seq_len, int sink,
     int ring_rows, const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
-    int n_new, int hkv, int chunks_per_row) {
+    int n_new, int hkv, int chunks_per_row, unsigned* status) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
@@ -145,6 +148,7 @@ __global__ void __launch_bounds__(256) kv_append_ring_fused_kernel(
       const int kvh = rest % hkv;
       const int tok = rest / hkv;
       const int slot = ring_slot(start + tok, sink, ring_rows);
+      if (!FLUX_IN_BOUNDS(slot >= 0 && slot < rows, status)) continue;
       const size_t dst = ((size_t(b) * hkv + kvh) * rows + slot) * row_elems + ch * 8;
       *reinterpret_cast<uint4*>(k_ring + dst) = __ldg(ks + i);
       *reinterpret_cast<uint4*>(v_ring + dst) = __ldg(vs + i);
@@ -185,6 +189,7 @@ __global__ void __launch_bounds__(256) kv_compact_ring_kernel(
     const int kvh = int(rest % hkv);
     const int r = int(rest / hkv);
     const int pos = r < head ? r : tail0 + (r - head);
+    if (!FLUX_IN_BOUNDS(pos >= 0 && pos < capacity, status)) continue;
     const size_t src = ((size_t(b) * hkv + kvh) * capacity + pos) * row_elems + ch * 8;
     const size_t dst =
         ((size_t(b) * hkv + kvh) * rows + ring_slot(pos, sink, ring_rows)) * row_elems + ch * 8;
@@ -201,18 +206,19 @@ constexpr long long kFusedAppendChunks = 4096;
 cudaError_t launch_kv_append_ring(const AttnGeom& g, uint16_t* k_ring, uint16_t* v_ring,
                                   int32_t* seq_len, int batch, int ring_rows,
                                   const uint16_t* k_new, const uint16_t* v_new, int n_new,
-                                  cudaStream_t stream) {
+                                  unsigned* status, cudaStream_t stream) {
   const int chunks = g.head_dim / 8;
   const long long per_seq = (long long)n_new * g.hkv * chunks;
   if (per_seq <= kFusedAppendChunks)
     return launch_pdl(kv_append_ring_fused_kernel, dim3(batch), dim3(256), 0, stream, k_ring,
-                      v_ring, seq_len, g.sink, ring_rows, k_new, v_new, n_new, g.hkv, chunks);
+                      v_ring, seq_len, g.sink, ring_rows, k_new, v_new, n_new, g.hkv, chunks,
+                      status);
   long long blocks = (per_seq + 255) / 256;
   const long long cap_blocks = (long long)device_sm_count() * 16 / (batch > 0 ? batch : 1) + 1;
   if (blocks > cap_blocks) blocks = cap_blocks;
   if (blocks < 1) blocks = 1;
   kv_append_ring_kernel<<<dim3(unsigned(blocks), batch), 256, 0, stream>>>(
-      k_ring, v_ring, seq_len, g.sink, ring_rows, k_new, v_new, n_new, g.hkv, chunks);
+      k_ring, v_ring, seq_len, g.sink, ring_rows, k_new, v_new, n_new, g.hkv, chunks, status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   kv_advance_unbounded_kernel<<<(batch + 127) / 128, 128, 0, stream>>>(seq_len, batch, n_new);

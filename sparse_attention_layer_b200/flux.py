@@ -5,6 +5,9 @@ Every function takes torch tensors that already live on the GPU, checks dtype,
 device, contiguity and shape, and passes raw pointers, sizes and the current CUDA
 stream to the library.  All arithmetic runs in the library's kernels; there is no
 CPU fallback: if libflux.so is missing or cannot load, every call raises.
+
+With FLUX_CHECKED=1 in the environment the binding loads libflux_checked.so instead:
+the same kernels with their bounds guards compiled in (include/flux.h).
 """
 
 from __future__ import annotations
@@ -15,7 +18,9 @@ from dataclasses import dataclass
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libflux.so")
+_LIB_PATH = os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "lib",
+    "libflux_checked.so" if os.environ.get("FLUX_CHECKED") == "1" else "libflux.so")
 
 FLUX_OK = 0
 FLUX_ERR_INVALID_ARG = 1
@@ -30,6 +35,7 @@ FLUX_DEVICE_TIMEOUT = 0x2
 FLUX_DEVICE_BAD_LENGTH = 0x4
 FLUX_DEVICE_RING_ROUTE = 0x8
 FLUX_DEVICE_LAYOUT = 0x10
+FLUX_DEVICE_BOUNDS = 0x20
 
 # every entry point declared in include/flux.h
 EXPORTED = (
@@ -38,7 +44,7 @@ EXPORTED = (
     "flux_get_device_status", "flux_status_string", "flux_version", "flux_decode_static",
     "flux_kv_compact_ring", "flux_kv_append_ring", "flux_decode_ring",
     "flux_selftest_wait_timeout", "flux_prefill_tile_plan", "flux_decode_append",
-    "flux_decode_append_ring",
+    "flux_decode_append_ring", "flux_selftest_bounds", "flux_build_checked",
 )
 
 # flag bit of a flux_prefill_tile_plan entry: the kernel masks keys of that tile
@@ -146,6 +152,10 @@ def lib() -> ctypes.CDLL:
         L.flux_decode_ring.restype = ctypes.c_int
         L.flux_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         L.flux_selftest_wait_timeout.restype = ctypes.c_int
+        L.flux_selftest_bounds.argtypes = [vp]
+        L.flux_selftest_bounds.restype = ctypes.c_int
+        L.flux_build_checked.argtypes = []
+        L.flux_build_checked.restype = ctypes.c_int
         L.flux_prefill_tile_plan.argtypes = [ctypes.POINTER(FluxAttnCfg), i32, vp, vp, i32, i32,
                                              i32, vp, i32, vp]
         L.flux_prefill_tile_plan.restype = ctypes.c_int
@@ -401,6 +411,17 @@ def flux_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     """Launch a wait that nothing releases; it must time out into FLUX_DEVICE_TIMEOUT."""
     _check("flux_selftest_wait_timeout",
            lib().flux_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def flux_selftest_bounds(stream=None) -> None:
+    """Launch a bounds guard that refuses its index: FLUX_DEVICE_BOUNDS in the checked
+    build, no status bit in the plain build."""
+    _check("flux_selftest_bounds", lib().flux_selftest_bounds(_stream(stream)))
+
+
+def flux_build_checked() -> bool:
+    """True when the loaded library is the checked build."""
+    return bool(lib().flux_build_checked())
 
 
 def flux_sa_block_ranges(cfg: AttnCfg, n_qblocks: int, ranges, stream=None) -> None:

@@ -51,6 +51,20 @@ def test_library_exports_every_header_symbol(L):
         assert hasattr(L, name), f"libflux.so does not export {name}"
 
 
+def test_checked_build_exports_the_same_entry_points(L):
+    """libflux_checked.so (bounds guards compiled in) builds here too, exports every
+    header symbol, and says which build it is; the plain library says it is not."""
+    path = build.build(checked=True)
+    assert path.endswith("libflux_checked.so")
+    C = ctypes.CDLL(path)
+    for name in header_functions():
+        assert hasattr(C, name), f"libflux_checked.so does not export {name}"
+    C.flux_build_checked.restype = ctypes.c_int
+    L.flux_build_checked.restype = ctypes.c_int
+    assert C.flux_build_checked() == 1
+    assert L.flux_build_checked() == 0
+
+
 def test_library_is_sm100a_only(L):
     # the build passes exactly one -gencode, for sm_100a
     assert build.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
