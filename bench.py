@@ -378,9 +378,11 @@ class PrefillBench:
         for c in self.model.caches:
             c.seq_len.zero_()
 
-    def step(self, route=True, fa_events=None, sa_events=None, router_events=None):
+    def step(self, route=True, fa_events=None, sa_events=None, router_events=None,
+             append_events=None):
         """router (optional) + every layer's KV append and prefill; with *_events, the
-        FA / SA prefill launches and the router are bracketed by CUDA events."""
+        FA / SA prefill launches, the appends and the router are bracketed by CUDA
+        events."""
         from sparse_attention_layer_b200 import flux
         m, w = self.model, self.w
 
@@ -396,7 +398,13 @@ class PrefillBench:
                 router_events.append((e0, e1))
         for layer in range(w.n_layers):
             c = m.caches[layer]
+            if append_events is not None:
+                a0, a1 = ev(), ev()
+                a0.record()
             flux.flux_kv_append(self.cfg, c.k, c.v, c.seq_len, self.k, self.v)
+            if append_events is not None:
+                a1.record()
+                append_events.append((a0, a1))
             events = fa_events if self.fa[layer] else sa_events
             if events is not None:
                 e0, e1 = ev(), ev()
@@ -709,7 +717,7 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
         pb.reset()
         pb.step()
     n_pf = max(3, min(10, args.steps))
-    pf_ms, fa_ev, sa_ev, rt_ev = [], [], [], []
+    pf_ms, fa_ev, sa_ev, rt_ev, ap_ev = [], [], [], [], []
     sampler = ClockSampler(local).start()
     barrier(world)
     for _ in range(n_pf):
@@ -717,7 +725,7 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
-        pb.step(fa_events=fa_ev, sa_events=sa_ev, router_events=rt_ev)
+        pb.step(fa_events=fa_ev, sa_events=sa_ev, router_events=rt_ev, append_events=ap_ev)
         b.record()
         pf_ms.append((a, b))
     barrier(world)
@@ -803,6 +811,13 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
         "roofline_sa": tensor_roofline("prefill_kernel<128> (tcgen05), SA layers", flops_sa,
                                        statistics.mean(elapsed_ms(sa_ev)), peaks, peak_kind,
                                        clocks, traffic=measured_traffic("prefill_sa", w.batch)),
+        # the layer's KV append: the prompt's K and V rows read from the projection layout
+        # and written head-major into the cache (a copy: the measured peak's own kind)
+        "append_roofline": hbm_roofline(
+            "kv_append_copy_kernel + kv_append_advance_kernel (flux_kv_append, one layer)",
+            2.0 * 2 * w.batch * w.seq * w.n_kv_heads * w.head_dim * 2,
+            statistics.mean(elapsed_ms(ap_ev)), peaks, peak_kind,
+            timing="CUDA events around each layer's flux_kv_append inside the timed steps"),
         "routing_mix": mix,
         "e2e": e2e,
         "gpu_launches_per_step": pb.launches_per_step,
