@@ -827,7 +827,7 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
     del pb, xq_h, q_h, k_h, v_h, o_h
     torch.cuda.empty_cache()
     if world == 1 and not args.no_cpu:
-        out["cpu_baseline"] = cpu_prefill_baseline(w, n_fa, n_rows=1024)
+        out["cpu_baseline"] = cpu_prefill_baseline(w, n_fa, n_rows=2048)
     return out
 
 
@@ -876,7 +876,7 @@ def run_prefill_qwen(args, world, local, peaks, peak_kind):
     del pb
     torch.cuda.empty_cache()
     if world == 1 and not args.no_cpu:
-        out["cpu_baseline"] = cpu_prefill_baseline(w, n_fa, n_rows=32)
+        out["cpu_baseline"] = cpu_prefill_baseline(w, n_fa, n_rows=64)
     return out
 
 
@@ -1051,10 +1051,10 @@ def run_flux(args, world, rank, local):
     if world == 1 and rank == 0 and not args.no_cpu:
         w, _ = decode_geometry()
         t0 = time.perf_counter()
-        tok_s, _ = cpu_baseline_decode_tok_s(w, len(dec["sa_layers"]), n_seq=2, chunks=6)
+        tok_s, _ = cpu_baseline_decode_tok_s(w, len(dec["sa_layers"]), n_seq=2, chunks=8)
         cpu = {"value": tok_s, "unit": "tokens/s", "cores": host_cores(),
                "blas_threads": blas_threads(), "kind": "oracle", "extrapolated": True,
-               "sample": "one decode token of 12 sequences (6 draws of 2) at 32768 context for "
+               "sample": "one decode token of all 16 sequences (8 draws of 2) at 32768 context for "
                          "one FA and one SA layer (fp64 oracle), scaled to 16 FA + 16 SA "
                          f"layers; {time.perf_counter() - t0:.1f} s wall, data generation "
                          "included"}
