@@ -32,7 +32,7 @@ cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
 }
 
-// ----- decode (split-KV + combine)
+// ----- decode (split-KV; split pairs are merged inside the same launch)
 constexpr int kDecMaxSplits = 64;   // splits per (sequence, KV head)
 constexpr int kDecStageKeys = 128;  // keys per decode pipeline stage
 constexpr int kDecMaxBatch = 1024;
