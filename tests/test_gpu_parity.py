@@ -377,6 +377,18 @@ def test_prefill_qwen_full_size(fa):
                   capacity=w.seq)
 
 
+@pytest.mark.parametrize("fa", [True, False])
+def test_prefill_llama_128k(fa):
+    """The sweep's longest prefill point in the Llama geometry (block 128, sink 128,
+    window 2048): a 131072-token prompt, sampled rows."""
+    w = configs.LLAMA_PREFILL
+    cfg = cfg_of(w)
+    seq = 131072
+    rows = sample_rows(seq, 0, cfg, 16, seed=3)
+    _prefill_case(cfg, [0], seq, [fa], seed=950 + fa, rows=rows, heads=[0, 31],
+                  capacity=seq)
+
+
 def test_decode_llama_full_size():
     """Llama-3.1-8B decode: 16 sequences at 32768 context, FA and SA layers."""
     w = configs.LLAMA_DECODE
