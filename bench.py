@@ -803,6 +803,8 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
                     f"(seeded; {w.n_layers - n_fa} SA layers), SA sink 128 + window 2048",
         "tokens_per_s": world * w.batch * w.seq / (pf_step / 1e3),
         "ms_per_step": pf_step, "steps": n_pf, "sa_layers": w.n_layers - n_fa,
+        # the router's sparsity ratio: the share of layers it sends to SA
+        "omega_msr": (w.n_layers - n_fa) / w.n_layers,
         "router_ms": statistics.mean(elapsed_ms(rt_ev)),
         "algorithmic_tflops_per_step": (n_fa * flops_fa + (w.n_layers - n_fa) * flops_sa) / 1e12,
         "roofline": tensor_roofline("prefill_kernel<128> (tcgen05), FA layers", flops_fa,
@@ -863,7 +865,8 @@ def run_prefill_qwen(args, world, local, peaks, peak_kind):
         "workload": "qwen3-4b-shape prefill, 1 x 131072 tokens, 36 layers, router 2560->256->36 "
                     f"(seeded; {w.n_layers - n_fa} SA layers), SA sink 128 + window 4096",
         "tokens_per_s": world * w.batch * w.seq / (ms / 1e3), "ms_per_step": ms, "steps": 2,
-        "sa_layers": w.n_layers - n_fa, "router_ms": statistics.mean(elapsed_ms(rt_ev)),
+        "sa_layers": w.n_layers - n_fa, "omega_msr": (w.n_layers - n_fa) / w.n_layers,
+        "router_ms": statistics.mean(elapsed_ms(rt_ev)),
         "fa_layer_ms": statistics.mean(elapsed_ms(fa_ev)),
         "sa_layer_ms": statistics.mean(elapsed_ms(sa_ev)),
         "algorithmic_tflops_per_step": (n_fa * flops_fa + (w.n_layers - n_fa) * flops_sa) / 1e12,
