@@ -1036,6 +1036,119 @@ def run_sweep_subset():
                     "fewer distinct caches than layers (the full model does not fit)"}
 
 
+def run_table16():
+    """The pages' latency-memory comparison (Table 16: Omega_MSR, prefill ms, decode
+    ms/token, persistent KV GiB and its saving, peak GiB, at 8K and 16K contexts) for
+    this attention path: Llama-3.1-8B shape, batch 1, routes from the seeded router on
+    synthetic x_Q, against every layer on FA (the dense reference).  Memory counts what
+    the attention path holds on the device (KV caches, q/k/v/o, x_Q, workspace), not a
+    model's weights or activations."""
+    import dataclasses
+
+    from sparse_attention_layer_b200 import configs, inputs
+    from sparse_attention_layer_b200.runtime import DecodeStepGraph, HybridAttention
+    GiB = float(1 << 30)
+    out = {}
+    for T in (8192, 16384):
+        w = dataclasses.replace(configs.LLAMA_PREFILL, seq=T)
+        cfg = llama_sweep_cfg()
+        base_alloc = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        steps = 48
+        model = HybridAttention(cfg, 1, T + steps + 16, "cuda")
+        router = [t.cuda() for t in inputs.router_weights(w.router_hidden, w.router_rank,
+                                                            w.n_layers, w.router_seed)]
+        xq = inputs.normal_bf16((1, T, w.router_hidden),
+                                inputs.layer_seed(w.data_seed, 0, inputs.XQ)).cuda()
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(1600 + T)
+        q = torch.randn(1, T, cfg.n_q_heads, cfg.head_dim, device="cuda",
+                        generator=gen).to(torch.bfloat16)
+        k = torch.randn(1, T, cfg.n_kv_heads, cfg.head_dim, device="cuda",
+                        generator=gen).to(torch.bfloat16)
+        v = torch.randn_like(k)
+        o = torch.empty_like(q)
+        L = cfg.n_layers
+        dq = torch.randn(L, 1, cfg.n_q_heads, cfg.head_dim, device="cuda").to(torch.bfloat16)
+        dk = torch.randn(L, 1, 1, cfg.n_kv_heads, cfg.head_dim, device="cuda").to(torch.bfloat16)
+        dv = torch.randn_like(dk)
+        do = torch.empty_like(dq)
+        model.route(*router, xq, w.pool_len, w.tau)
+        router_mask = model.fa_mask.clone()
+        all_fa = inputs.pack_bits_u32(inputs.fa_bits_from_sa_layers(1, L, [])).cuda()
+
+        def prefill(route):
+            for c in model.caches:
+                c.seq_len.zero_()
+            if route:
+                model.route(*router, xq, w.pool_len, w.tau)
+            for layer in range(L):
+                model.prefill_layer(layer, q, k, v, o)
+
+        def timed(fn, reps=3):
+            fn()
+            times = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                times.append((a, b))
+            torch.cuda.synchronize()
+            return statistics.median(x.elapsed_time(y) for x, y in times)
+
+        def decode_ms():
+            # one eager step (library set-up), then the captured step, replayed; the
+            # appends advance the lengths from T
+            for layer in range(L):
+                model.decode_layer(layer, dq[layer], dk[layer], dv[layer], do[layer])
+            g = DecodeStepGraph(model, dq, dk, dv, do)
+            ms = graph_ms(g.graph, warm=3, reps=20)
+            del g
+            return ms
+
+        model.set_mask(all_fa)
+        row_fa_prefill = timed(lambda: prefill(False))
+        prefill(False)
+        row_fa_decode = decode_ms()
+        peak_prefill = (torch.cuda.max_memory_allocated() - base_alloc) / GiB
+        kv_fa = model.kv_bytes() / GiB
+        model.set_mask(router_mask)
+        row_flux_prefill = timed(lambda: prefill(True))
+        prefill(False)
+        n_sa = len(model.sa_layers())
+        row_flux_decode = decode_ms()
+        model.evict_sa_layers()
+        torch.cuda.synchronize()
+        kv_flux = model.kv_bytes() / GiB
+        row_flux_decode_rings = decode_ms()
+        # the context's own K/V (T rows per layer; the allocation adds room for the steps)
+        per_row = 2 * cfg.n_kv_heads * cfg.head_dim * 2
+        logical_full = L * T * per_row / GiB
+        logical_flux = ((L - n_sa) * T + n_sa * (cfg.sink + cfg.window)) * per_row / GiB
+        row = {
+            "omega_msr": n_sa / L, "sa_layers": n_sa,
+            "prefill_ms": {"flux": row_flux_prefill, "all_fa": row_fa_prefill,
+                           "speedup": row_fa_prefill / row_flux_prefill},
+            "decode_ms_per_token": {"flux": row_flux_decode, "all_fa": row_fa_decode,
+                                    "speedup": row_fa_decode / row_flux_decode,
+                                    "flux_sa_layers_evicted": row_flux_decode_rings},
+            "persistent_kv_gib": {"all_fa": logical_full, "flux_evicted": logical_flux,
+                                  "saving": 1.0 - logical_flux / logical_full,
+                                  "allocated_all_fa": kv_fa, "allocated_flux_evicted": kv_flux},
+            "peak_gib_prefill": peak_prefill,
+        }
+        out[f"{T // 1024}K"] = row
+        del model, xq, q, k, v, o, dq, dk, dv, do
+        torch.cuda.empty_cache()
+    out["what"] = ("batch 1, Llama-3.1-8B attention shape, seeded router on synthetic x_Q "
+                   "(routes) vs all layers on FA; prefill = router + 32 x (append + prefill); "
+                   "decode = the captured 32-layer step (one token); persistent KV = the "
+                   "context's K/V rows, SA layers as rings of sink + window rows after "
+                   "eviction; peak = device memory the attention path allocated")
+    return out
+
+
 def run_flux(args, world, rank, local):
     from sparse_attention_layer_b200 import flux
     peaks, peak_kind = load_peaks()
@@ -1046,6 +1159,7 @@ def run_flux(args, world, rank, local):
         extra["prefill_qwen_128k"] = run_prefill_qwen(args, world, local, peaks, peak_kind)
         extra["pages_sa_geometry"] = run_pages_geometry(peaks, peak_kind)
         extra["sweep_subset"] = run_sweep_subset()
+        extra["table16_llama"] = run_table16()
     if flux.flux_get_device_status():
         raise RuntimeError("device status set during the benchmark")
 
