@@ -819,6 +819,7 @@ def run_prefill_llama(args, world, local, peaks, peak_kind):
             "kv_append_copy_kernel + kv_append_advance_kernel (flux_kv_append, one layer)",
             2.0 * 2 * w.batch * w.seq * w.n_kv_heads * w.head_dim * 2,
             statistics.mean(elapsed_ms(ap_ev)), peaks, peak_kind,
+            traffic=measured_traffic("append", w.batch),
             timing="CUDA events around each layer's flux_kv_append inside the timed steps"),
         "routing_mix": mix,
         "e2e": e2e,
