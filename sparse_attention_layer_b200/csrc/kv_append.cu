@@ -7,7 +7,8 @@
 //
 // Large appends (prefill) take two launches: the copy reads seq_len[b] as the write
 // position; the second launch advances seq_len[b], so no copy CTA can observe a
-// half-updated length.  Small appends (decode: a few rows per sequence) take one: a
+// half-updated length.  Both use programmatic dependent launch, so the second grid is
+// already scheduled when the first completes.  Small appends (decode: a few rows per sequence) take one: a
 // single CTA per sequence copies its rows and then advances seq_len[b] itself after a
 // CTA barrier; it is launched with programmatic dependent launch, like the decode
 // kernels after it.  A sequence that would pass the capacity is skipped and
@@ -28,6 +29,8 @@ __global__ void __launch_bounds__(256) kv_append_copy_kernel(
     const int32_t* __restrict__ seq_len, int capacity, const uint16_t* __restrict__ k_new,
     const uint16_t* __restrict__ v_new, int n_new, int hkv, int chunks_per_row,
     unsigned* status) {
+  pdl_trigger();  // the length update may be scheduled; it waits for this grid
+  pdl_wait();     // seq_len and the new rows may come from earlier kernels
   const int b = blockIdx.y;
   const int start = seq_len[b];
   if (start < 0 || start + n_new > capacity) {
@@ -87,6 +90,8 @@ __global__ void __launch_bounds__(256) kv_append_fused_kernel(
 }
 
 __global__ void kv_append_advance_kernel(int32_t* seq_len, int batch, int capacity, int n_new) {
+  pdl_trigger();
+  pdl_wait();  // every copy CTA has read its start (the copy grid has completed)
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
   const int start = seq_len[b];
@@ -254,13 +259,14 @@ cudaError_t launch_kv_append(const AttnGeom& g, uint16_t* k_cache, uint16_t* v_c
   const long long cap_blocks = (long long)device_sm_count() * 16 / (batch > 0 ? batch : 1) + 1;
   if (blocks > cap_blocks) blocks = cap_blocks;
   if (blocks < 1) blocks = 1;
-  kv_append_copy_kernel<<<dim3(unsigned(blocks), batch), 256, 0, stream>>>(
-      k_cache, v_cache, seq_len, capacity, k_new, v_new, n_new, g.hkv, chunks, status);
-  cudaError_t err = cudaGetLastError();
+  // both launches with programmatic dependent launch: each grid is scheduled while the
+  // one before it drains and waits (griddepcontrol.wait) for it to complete
+  cudaError_t err = launch_pdl(kv_append_copy_kernel, dim3(unsigned(blocks), batch), dim3(256),
+                               0, stream, k_cache, v_cache, seq_len, capacity, k_new, v_new,
+                               n_new, g.hkv, chunks, status);
   if (err != cudaSuccess) return err;
-  kv_append_advance_kernel<<<(batch + 127) / 128, 128, 0, stream>>>(seq_len, batch, capacity,
-                                                                     n_new);
-  return cudaGetLastError();
+  return launch_pdl(kv_append_advance_kernel, dim3((batch + 127) / 128), dim3(128), 0, stream,
+                    seq_len, batch, capacity, n_new);
 }
 
 }  // namespace flux
